@@ -1,0 +1,194 @@
+"""ctypes front end of the fp64 CPU oracle for the QSA MQA indexer score.
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU
+baseline use it; the product package never imports it.  All arrays are numpy
+(bf16 data travels as uint16 bit patterns) and everything runs on the host.
+What each function computes, and the passages it follows, is stated in
+``qsa_oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_i64, _int, _f64, _vp = C.c_int64, C.c_int, C.c_double, C.c_void_p
+
+SCALE = 1.0 / np.sqrt(128.0)
+
+
+def _bind(L: C.CDLL) -> C.CDLL:
+    L.qsa_oracle_default_threads.restype = _int
+    L.qsa_oracle_logical_position.restype = _i64
+    L.qsa_oracle_logical_position.argtypes = [_i64, _i64, _i64]
+    L.qsa_oracle_visible_blocks.restype = _i64
+    L.qsa_oracle_visible_blocks.argtypes = [_i64, _i64]
+    L.qsa_oracle_decode_visible.argtypes = [_vp, _i64, _i64, _vp]
+    L.qsa_oracle_prefill_intervals.argtypes = [_vp, _vp, _vp, _i64, _vp, _vp]
+    L.qsa_oracle_decode.argtypes = [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _i64, _i64,
+                                    _vp, _i64, _i64, _vp, _i64, _i64, _f64, _vp, _i64, _int]
+    L.qsa_oracle_decode_entries.argtypes = [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _i64, _i64,
+                                            _vp, _i64, _i64, _vp, _i64, _i64, _f64,
+                                            _vp, _vp, _vp, _i64, _vp, _int]
+    L.qsa_oracle_prefill.argtypes = [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f64,
+                                     _vp, _i64, _int]
+    L.qsa_oracle_prefill_entries.argtypes = [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _f64,
+                                             _vp, _vp, _i64, _vp, _int]
+    L.qsa_oracle_topk.argtypes = [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _int]
+    return L
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def _bf16_bits(x) -> tuple[np.ndarray, tuple[int, ...]]:
+    """bf16 tensor/array -> (uint16 bit array, element strides)."""
+    if hasattr(x, "view") and hasattr(x, "dtype") and str(x.dtype) == "torch.bfloat16":
+        import torch
+        x = x.detach().cpu()
+        bits = x.view(torch.int16).numpy().view(np.uint16)
+        return bits, tuple(x.stride())
+    a = np.asarray(x)
+    if a.dtype != np.uint16:
+        raise TypeError("bf16 data must be a torch.bfloat16 tensor or uint16 bit array")
+    return a, tuple(s // 2 for s in a.strides)
+
+
+def _i32(x) -> np.ndarray:
+    a = x.cpu().numpy() if hasattr(x, "cpu") else np.asarray(x)
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+class Oracle:
+    """One loaded build of the oracle library."""
+
+    def __init__(self, path: str | None = None):
+        self.L = _bind(C.CDLL(path or _build.build()))
+
+    def default_threads(self) -> int:
+        return int(self.L.qsa_oracle_default_threads())
+
+    def visible_blocks(self, pos: int, seq_len: int) -> int:
+        return int(self.L.qsa_oracle_visible_blocks(pos, seq_len))
+
+    def logical_position(self, seq_len: int, query_len: int, i: int) -> int:
+        return int(self.L.qsa_oracle_logical_position(seq_len, query_len, i))
+
+    def decode_visible(self, seq_lens, Q: int) -> np.ndarray:
+        """visible[b, i] of every decode row."""
+        sl = _i32(seq_lens)
+        out = np.zeros((sl.shape[0], Q), dtype=np.int32)
+        self.L.qsa_oracle_decode_visible(_ptr(sl), sl.shape[0], Q, _ptr(out))
+        return out
+
+    def prefill_intervals(self, cu_seqlens_q, seq_lens, key_offsets):
+        """(ks, ke) int32 [T] of a packed prefill batch."""
+        cu, sl, ko = _i32(cu_seqlens_q), _i32(seq_lens), _i32(key_offsets)
+        T = int(cu[-1])
+        ks = np.zeros(T, dtype=np.int32)
+        ke = np.zeros(T, dtype=np.int32)
+        self.L.qsa_oracle_prefill_intervals(_ptr(cu), _ptr(sl), _ptr(ko), sl.shape[0],
+                                            _ptr(ks), _ptr(ke))
+        return ks, ke
+
+    @staticmethod
+    def _decode_common(q, k_cache, page_table, seq_lens):
+        qb, qs = _bf16_bits(q)
+        kb, kst = _bf16_bits(k_cache)
+        if len(qs) != 4 or qs[3] != 1:
+            raise ValueError("q must be [B, Q, 4, 128] with unit feature stride")
+        if len(kst) != 4 or kst[3] != 1:
+            raise ValueError("k_cache must be [pages, page_size, 1, 128] with unit feature stride")
+        return qb, qs, kb, kst, _i32(page_table), _i32(seq_lens)
+
+    def decode(self, q, k_cache, page_table, seq_lens, W: int, scale: float = SCALE,
+               threads: int = 0) -> np.ndarray:
+        """fp64 scores [B, Q, W] of the paged decode / spec-decode path."""
+        qb, qs, kb, kst, pt, sl = self._decode_common(q, k_cache, page_table, seq_lens)
+        B, Q = qb.shape[0], qb.shape[1]
+        out = np.empty((B, Q, W), dtype=np.float64)
+        self.L.qsa_oracle_decode(_ptr(qb), qs[0], qs[1], qs[2], _ptr(kb), kb.shape[0],
+                                 kb.shape[1], kst[0], kst[1], _ptr(pt), pt.shape[1],
+                                 pt.shape[1], _ptr(sl), B, Q, float(scale), _ptr(out), W,
+                                 threads)
+        return out
+
+    def decode_entries(self, q, k_cache, page_table, seq_lens, b, i, n, scale: float = SCALE,
+                       threads: int = 0) -> np.ndarray:
+        """fp64 scores of the listed decode entries (row (b[e], i[e]), column n[e])."""
+        qb, qs, kb, kst, pt, sl = self._decode_common(q, k_cache, page_table, seq_lens)
+        bb = np.ascontiguousarray(b, dtype=np.int64)
+        ii = np.ascontiguousarray(i, dtype=np.int64)
+        nn = np.ascontiguousarray(n, dtype=np.int64)
+        out = np.empty(bb.shape[0], dtype=np.float64)
+        self.L.qsa_oracle_decode_entries(_ptr(qb), qs[0], qs[1], qs[2], _ptr(kb), kb.shape[0],
+                                         kb.shape[1], kst[0], kst[1], _ptr(pt), pt.shape[1],
+                                         pt.shape[1], _ptr(sl), qb.shape[0], qb.shape[1],
+                                         float(scale), _ptr(bb), _ptr(ii), _ptr(nn),
+                                         bb.shape[0], _ptr(out), threads)
+        return out
+
+    @staticmethod
+    def _prefill_common(q, k, ks, ke):
+        qb, qs = _bf16_bits(q)
+        kb, kst = _bf16_bits(k)
+        if len(qs) != 3 or qs[2] != 1:
+            raise ValueError("q must be [T, 4, 128] with unit feature stride")
+        if len(kst) != 2 or kst[1] != 1:
+            raise ValueError("k must be [Nk, 128] with unit feature stride")
+        return qb, qs, kb, kst, _i32(ks), _i32(ke)
+
+    def prefill(self, q, k, ks, ke, W: int, scale: float = SCALE, threads: int = 0) -> np.ndarray:
+        """fp64 scores [T, W] of the packed prefill path (column j holds key ks[t] + j)."""
+        qb, qs, kb, kst, a, b = self._prefill_common(q, k, ks, ke)
+        T = qb.shape[0]
+        out = np.empty((T, W), dtype=np.float64)
+        self.L.qsa_oracle_prefill(_ptr(qb), qs[0], qs[1], _ptr(kb), kst[0], kb.shape[0],
+                                  _ptr(a), _ptr(b), T, float(scale), _ptr(out), W, threads)
+        return out
+
+    def prefill_entries(self, q, k, ks, ke, t, j, scale: float = SCALE,
+                        threads: int = 0) -> np.ndarray:
+        """fp64 scores of the listed prefill entries (row t[e], column j[e])."""
+        qb, qs, kb, kst, a, b = self._prefill_common(q, k, ks, ke)
+        tt = np.ascontiguousarray(t, dtype=np.int64)
+        jj = np.ascontiguousarray(j, dtype=np.int64)
+        out = np.empty(tt.shape[0], dtype=np.float64)
+        self.L.qsa_oracle_prefill_entries(_ptr(qb), qs[0], qs[1], _ptr(kb), kst[0],
+                                          kb.shape[0], _ptr(a), _ptr(b), float(scale),
+                                          _ptr(tt), _ptr(jj), tt.shape[0], _ptr(out), threads)
+        return out
+
+    def topk(self, scores, lengths, k: int, threads: int = 0) -> np.ndarray:
+        """Column indices [rows, k] of the k largest scores among each row's first
+        lengths[r] columns, ascending, ties to the lower column, -1 padded."""
+        s = np.ascontiguousarray(scores, dtype=np.float64)
+        ln = _i32(lengths)
+        rows = s.shape[0]
+        if ln.shape[0] != rows or (rows and ln.max(initial=0) > s.shape[1]):
+            raise ValueError("lengths must have one entry per row and not exceed the row width")
+        idx = np.empty((rows, k), dtype=np.int32)
+        self.L.qsa_oracle_topk(_ptr(s), s.shape[1], _ptr(ln), rows, k, _ptr(idx), k, threads)
+        return idx
+
+
+_default: Oracle | None = None
+
+
+def get() -> Oracle:
+    """The oracle built from ``qsa_oracle.c`` (compiled on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+def __getattr__(name):
+    # module-level shortcuts: oracle.decode(...), oracle.topk(...), ...
+    if name.startswith("_"):
+        raise AttributeError(name)
+    return getattr(get(), name)

@@ -1,0 +1,315 @@
+/*
+ * QSA MQA indexer score: CPU oracle in fp64.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file; only the tests, the smoke check and the benchmark's CPU
+ * baseline do.  It shares no code, header or table with the CUDA path.
+ *
+ * What it computes, written out plainly (no tiling, no reordering):
+ *
+ *   score(t, n) = scale * sum_{h<4} max(0, sum_{c<128} q[t,h,c] * k[n,c])
+ *
+ * (QSA docs, MATE, section "MQA score": four query heads share one
+ * compressed key of dimension 128, the score sums the four head-wise ReLU
+ * dot products and scales by 1/sqrt(128), passed here as a multiplier.)
+ * bf16 inputs widen exactly to double and every sum runs in double, in index
+ * order.
+ *
+ * Masking (vLLM qsa_cache.py, "_logical_positions" and the metadata kernel's
+ * "visible_blocks"): a query token at logical position
+ *     pos = seq_len - query_len + i
+ * sees compressed keys n < visible = max(0, min((pos + 1) // 4, seq_len // 4));
+ * every other column is -inf.  Decode reads key n of request b from page
+ * page_table[b, n // page_size], row n % page_size (vLLM qsa_cache.py,
+ * "_logical_to_physical_qsa_slots"); an entry that is -1 or not a valid page
+ * gives -inf (QSA docs, "MQA score": missing or out-of-range pages are
+ * masked to -inf).  Prefill row t sees keys in its interval [ks[t], ke[t])
+ * clipped to [0, Nk); column j of the row holds key ks[t] + j.
+ *
+ * Parity status: every function here is pinned by the CPU tests (closed
+ * forms, invariants, exact integer brute force, the cache writer's rule and
+ * the FLOP counts printed in the vLLM PR's prefill table).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+#define QSA_HEADS 4
+#define QSA_DIM 128
+#define QSA_RATIO 4
+
+/* ---------------------------------------------------------------- helpers */
+
+static double bf16_to_double(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int64_t floor_div(int64_t a, int64_t b) {
+    int64_t q = a / b;
+    if ((a % b != 0) && ((a < 0) != (b < 0))) q -= 1;
+    return q;
+}
+
+/* A simple static split of [0, n) over threads. */
+typedef void (*range_fn)(void *ctx, int64_t begin, int64_t end);
+typedef struct { range_fn fn; void *ctx; int64_t begin, end; } range_job;
+
+static void *range_thread(void *arg) {
+    range_job *j = (range_job *)arg;
+    j->fn(j->ctx, j->begin, j->end);
+    return NULL;
+}
+
+int qsa_oracle_default_threads(void) {
+    long n = sysconf(_SC_NPROCESSORS_ONLN);
+    return n > 0 ? (int)n : 1;
+}
+
+static void parallel_for(int64_t n, int nthreads, range_fn fn, void *ctx) {
+    if (nthreads <= 0) nthreads = qsa_oracle_default_threads();
+    if (nthreads > n) nthreads = (int)(n > 0 ? n : 1);
+    if (nthreads <= 1) { fn(ctx, 0, n); return; }
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    range_job *jobs = (range_job *)malloc(sizeof(range_job) * (size_t)nthreads);
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i].fn = fn; jobs[i].ctx = ctx;
+        jobs[i].begin = n * i / nthreads;
+        jobs[i].end = n * (i + 1) / nthreads;
+        pthread_create(&th[i], NULL, range_thread, &jobs[i]);
+    }
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+    free(jobs);
+}
+
+/* ------------------------------------------------------------- the mask */
+
+int64_t qsa_oracle_logical_position(int64_t seq_len, int64_t query_len, int64_t i) {
+    return seq_len - query_len + i;
+}
+
+int64_t qsa_oracle_visible_blocks(int64_t pos, int64_t seq_len) {
+    int64_t by_pos = floor_div(pos + 1, QSA_RATIO);
+    int64_t by_len = floor_div(seq_len, QSA_RATIO);
+    int64_t v = by_pos < by_len ? by_pos : by_len;
+    return v > 0 ? v : 0;
+}
+
+/* visible[b * Q + i] for every decode row. */
+void qsa_oracle_decode_visible(const int32_t *seq_lens, int64_t B, int64_t Q, int32_t *visible) {
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t i = 0; i < Q; ++i) {
+            int64_t pos = qsa_oracle_logical_position(seq_lens[b], Q, i);
+            visible[b * Q + i] = (int32_t)qsa_oracle_visible_blocks(pos, seq_lens[b]);
+        }
+}
+
+/* Per-row key intervals of a packed prefill batch: sequence s has query rows
+ * cu_seqlens_q[s] .. cu_seqlens_q[s+1], seq_lens[s] tokens in all, and its
+ * keys start at key_offsets[s]. */
+void qsa_oracle_prefill_intervals(const int32_t *cu_seqlens_q, const int32_t *seq_lens,
+                                  const int32_t *key_offsets, int64_t S,
+                                  int32_t *ks, int32_t *ke) {
+    for (int64_t s = 0; s < S; ++s) {
+        int64_t qlen = (int64_t)cu_seqlens_q[s + 1] - cu_seqlens_q[s];
+        for (int64_t i = 0; i < qlen; ++i) {
+            int64_t t = cu_seqlens_q[s] + i;
+            int64_t pos = qsa_oracle_logical_position(seq_lens[s], qlen, i);
+            ks[t] = key_offsets[s];
+            ke[t] = (int32_t)(key_offsets[s] + qsa_oracle_visible_blocks(pos, seq_lens[s]));
+        }
+    }
+}
+
+/* ------------------------------------------------------------- the score */
+
+/* scale * sum_h max(0, q_h . k) for one query row (4 heads) and one key. */
+static double head_sum_score(const uint16_t *q_row, int64_t q_stride_h,
+                             const uint16_t *k_row, double scale) {
+    double s = 0.0;
+    for (int h = 0; h < QSA_HEADS; ++h) {
+        const uint16_t *qh = q_row + h * q_stride_h;
+        double d = 0.0;
+        for (int c = 0; c < QSA_DIM; ++c) d += bf16_to_double(qh[c]) * bf16_to_double(k_row[c]);
+        s += d > 0.0 ? d : 0.0;
+    }
+    return scale * s;
+}
+
+typedef struct {
+    const uint16_t *q; int64_t q_sb, q_st, q_sh;
+    const uint16_t *k_cache; int64_t num_pages, page_size, k_page_stride, k_row_stride;
+    const int32_t *page_table; int64_t pt_stride, max_pages;
+    const int32_t *seq_lens; int64_t B, Q;
+    double scale;
+} decode_args;
+
+/* Score of decode row (b, i) against compressed key n, or -inf when masked. */
+static double decode_entry(const decode_args *a, int64_t b, int64_t i, int64_t n) {
+    int64_t pos = qsa_oracle_logical_position(a->seq_lens[b], a->Q, i);
+    int64_t visible = qsa_oracle_visible_blocks(pos, a->seq_lens[b]);
+    if (n < 0 || n >= visible) return -INFINITY;
+    int64_t logical_page = n / a->page_size;
+    if (logical_page >= a->max_pages) return -INFINITY;
+    int64_t page = a->page_table[b * a->pt_stride + logical_page];
+    if (page < 0 || page >= a->num_pages) return -INFINITY;
+    const uint16_t *k_row = a->k_cache + page * a->k_page_stride + (n % a->page_size) * a->k_row_stride;
+    const uint16_t *q_row = a->q + b * a->q_sb + i * a->q_st;
+    return head_sum_score(q_row, a->q_sh, k_row, a->scale);
+}
+
+typedef struct { decode_args a; double *out; int64_t W; } decode_full_ctx;
+
+static void decode_rows(void *vctx, int64_t begin, int64_t end) {
+    decode_full_ctx *c = (decode_full_ctx *)vctx;
+    for (int64_t r = begin; r < end; ++r) {
+        int64_t b = r / c->a.Q, i = r % c->a.Q;
+        for (int64_t n = 0; n < c->W; ++n) c->out[r * c->W + n] = decode_entry(&c->a, b, i, n);
+    }
+}
+
+/* out[(b * Q + i) * W + n] for every row and every n < W. */
+void qsa_oracle_decode(const uint16_t *q, int64_t q_sb, int64_t q_st, int64_t q_sh,
+                       const uint16_t *k_cache, int64_t num_pages, int64_t page_size,
+                       int64_t k_page_stride, int64_t k_row_stride,
+                       const int32_t *page_table, int64_t pt_stride, int64_t max_pages,
+                       const int32_t *seq_lens, int64_t B, int64_t Q, double scale,
+                       double *out, int64_t W, int nthreads) {
+    decode_full_ctx c = {{q, q_sb, q_st, q_sh, k_cache, num_pages, page_size, k_page_stride,
+                          k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale},
+                         out, W};
+    parallel_for(B * Q, nthreads, decode_rows, &c);
+}
+
+typedef struct { decode_args a; const int64_t *bb, *ii, *nn; double *out; } decode_entries_ctx;
+
+static void decode_entries_range(void *vctx, int64_t begin, int64_t end) {
+    decode_entries_ctx *c = (decode_entries_ctx *)vctx;
+    for (int64_t e = begin; e < end; ++e) c->out[e] = decode_entry(&c->a, c->bb[e], c->ii[e], c->nn[e]);
+}
+
+/* out[e] = score of decode row (bb[e], ii[e]) at column nn[e]. */
+void qsa_oracle_decode_entries(const uint16_t *q, int64_t q_sb, int64_t q_st, int64_t q_sh,
+                               const uint16_t *k_cache, int64_t num_pages, int64_t page_size,
+                               int64_t k_page_stride, int64_t k_row_stride,
+                               const int32_t *page_table, int64_t pt_stride, int64_t max_pages,
+                               const int32_t *seq_lens, int64_t B, int64_t Q, double scale,
+                               const int64_t *bb, const int64_t *ii, const int64_t *nn,
+                               int64_t count, double *out, int nthreads) {
+    decode_entries_ctx c = {{q, q_sb, q_st, q_sh, k_cache, num_pages, page_size, k_page_stride,
+                             k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale},
+                            bb, ii, nn, out};
+    parallel_for(count, nthreads, decode_entries_range, &c);
+}
+
+typedef struct {
+    const uint16_t *q; int64_t q_st, q_sh;
+    const uint16_t *k; int64_t k_stride, Nk;
+    const int32_t *ks, *ke;
+    double scale;
+} prefill_args;
+
+/* Score of prefill row t at column j (key ks[t] + j), or -inf when masked. */
+static double prefill_entry(const prefill_args *a, int64_t t, int64_t j) {
+    int64_t lo = a->ks[t] > 0 ? a->ks[t] : 0;
+    int64_t hi = a->ke[t] < a->Nk ? a->ke[t] : a->Nk;
+    int64_t n = (int64_t)a->ks[t] + j;
+    if (j < 0 || n < lo || n >= hi) return -INFINITY;
+    return head_sum_score(a->q + t * a->q_st, a->q_sh, a->k + n * a->k_stride, a->scale);
+}
+
+typedef struct { prefill_args a; double *out; int64_t W; } prefill_full_ctx;
+
+static void prefill_rows(void *vctx, int64_t begin, int64_t end) {
+    prefill_full_ctx *c = (prefill_full_ctx *)vctx;
+    for (int64_t t = begin; t < end; ++t)
+        for (int64_t j = 0; j < c->W; ++j) c->out[t * c->W + j] = prefill_entry(&c->a, t, j);
+}
+
+/* out[t * W + j] for every row t < T and column j < W. */
+void qsa_oracle_prefill(const uint16_t *q, int64_t q_st, int64_t q_sh,
+                        const uint16_t *k, int64_t k_stride, int64_t Nk,
+                        const int32_t *ks, const int32_t *ke, int64_t T, double scale,
+                        double *out, int64_t W, int nthreads) {
+    prefill_full_ctx c = {{q, q_st, q_sh, k, k_stride, Nk, ks, ke, scale}, out, W};
+    parallel_for(T, nthreads, prefill_rows, &c);
+}
+
+typedef struct { prefill_args a; const int64_t *tt, *jj; double *out; } prefill_entries_ctx;
+
+static void prefill_entries_range(void *vctx, int64_t begin, int64_t end) {
+    prefill_entries_ctx *c = (prefill_entries_ctx *)vctx;
+    for (int64_t e = begin; e < end; ++e) c->out[e] = prefill_entry(&c->a, c->tt[e], c->jj[e]);
+}
+
+/* out[e] = score of prefill row tt[e] at column jj[e]. */
+void qsa_oracle_prefill_entries(const uint16_t *q, int64_t q_st, int64_t q_sh,
+                                const uint16_t *k, int64_t k_stride, int64_t Nk,
+                                const int32_t *ks, const int32_t *ke, double scale,
+                                const int64_t *tt, const int64_t *jj, int64_t count,
+                                double *out, int nthreads) {
+    prefill_entries_ctx c = {{q, q_st, q_sh, k, k_stride, Nk, ks, ke, scale}, tt, jj, out};
+    parallel_for(count, nthreads, prefill_entries_range, &c);
+}
+
+/* ------------------------------------------------------------- top-k */
+
+/* Per-row top-k (the caller's selection step in the QSA docs' pipeline;
+ * widths 512 / 1024 / 2048 in the vLLM PR's top-k discussion).  Among the
+ * first lengths[r] columns of row r, take the min(k, lengths[r]) largest
+ * scores, ties going to the lower column; write their column indices in
+ * ascending order and pad the rest of the k slots with -1.  -0.0 and +0.0
+ * compare equal.  The ordering is done by the C library's qsort. */
+
+typedef struct { double v; int64_t j; } scored_col;
+
+static int by_score_desc_then_col(const void *pa, const void *pb) {
+    const scored_col *a = (const scored_col *)pa, *b = (const scored_col *)pb;
+    if (a->v > b->v) return -1;
+    if (a->v < b->v) return 1;
+    return (a->j > b->j) - (a->j < b->j);
+}
+
+static int by_col(const void *pa, const void *pb) {
+    int32_t a = *(const int32_t *)pa, b = *(const int32_t *)pb;
+    return (a > b) - (a < b);
+}
+
+typedef struct {
+    const double *scores; int64_t stride;
+    const int32_t *lengths; int64_t k;
+    int32_t *idx; int64_t idx_stride;
+} topk_ctx;
+
+static void topk_rows(void *vctx, int64_t begin, int64_t end) {
+    topk_ctx *c = (topk_ctx *)vctx;
+    for (int64_t r = begin; r < end; ++r) {
+        int64_t len = c->lengths[r] > 0 ? c->lengths[r] : 0;
+        int32_t *dst = c->idx + r * c->idx_stride;
+        int64_t take = len < c->k ? len : c->k;
+        if (len > 0) {
+            scored_col *cols = (scored_col *)malloc(sizeof(scored_col) * (size_t)len);
+            for (int64_t j = 0; j < len; ++j) {
+                cols[j].v = c->scores[r * c->stride + j];
+                cols[j].j = j;
+            }
+            qsort(cols, (size_t)len, sizeof(scored_col), by_score_desc_then_col);
+            for (int64_t s = 0; s < take; ++s) dst[s] = (int32_t)cols[s].j;
+            free(cols);
+            qsort(dst, (size_t)take, sizeof(int32_t), by_col);
+        }
+        for (int64_t s = take; s < c->k; ++s) dst[s] = -1;
+    }
+}
+
+void qsa_oracle_topk(const double *scores, int64_t stride, const int32_t *lengths, int64_t rows,
+                     int64_t k, int32_t *idx, int64_t idx_stride, int nthreads) {
+    topk_ctx c = {scores, stride, lengths, k, idx, idx_stride};
+    parallel_for(rows, nthreads, topk_rows, &c);
+}

@@ -1,0 +1,365 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError
+when the oracle disagrees with:
+
+* the cache writer's rule (vLLM qsa_cache.py, "compressed_qsa_slot_mapping":
+  a token at logical position p writes compressed row p // 4 only when
+  (p + 1) % 4 == 0), simulated token by token;
+* the query positions of a decode step being the last Q tokens of the request;
+* the prefill FLOP counts printed in the vLLM PR "Separate prefill and decode
+  paths for QSA indexer" (section "Microbenchmarks", table "Prefill");
+* exact integer brute force on tiny inputs, done by another route (keys are
+  first gathered into a dense per-request list by walking the page table,
+  visibility comes from the writer simulation, sums are Python integers);
+* closed forms, invariants and cross-entry identities of the definition in
+  the QSA docs (MATE, section "MQA score");
+* a full sort for the top-k selection.
+
+The same functions run against deliberately broken builds of the oracle
+(``test_oracle_mutants.py``) to show that each plausible mistake trips a pin.
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+GOLDEN = os.path.join(HERE, "golden", "vllm_qsa_indexer_microbench.txt")
+SCALE = 1.0 / math.sqrt(128.0)
+
+
+# ---------------------------------------------------------------- helpers
+
+def keys_written_through(p: int) -> list[int]:
+    """Compressed rows in the cache once tokens 0..p have been processed."""
+    out = []
+    for tok in range(p + 1):
+        if (tok + 1) % 4 == 0:
+            out.append(tok // 4)
+    return out
+
+
+def int_bf16(shape, lo, hi, rng: np.random.Generator) -> torch.Tensor:
+    """Small integers, exactly representable in bf16."""
+    return torch.from_numpy(rng.integers(lo, hi + 1, size=shape).astype(np.float32)).to(torch.bfloat16)
+
+
+def as_int(x: torch.Tensor) -> np.ndarray:
+    return x.to(torch.float32).numpy().astype(np.int64)
+
+
+def int_score(q_row_heads: np.ndarray, k_row: np.ndarray) -> int:
+    """sum_h max(0, q_h . k) in exact integers (q_row_heads: [4, 128])."""
+    total = 0
+    for h in range(q_row_heads.shape[0]):
+        d = sum(int(a) * int(b) for a, b in zip(q_row_heads[h], k_row))
+        total += max(0, d)
+    return total
+
+
+def paged_case(rng, B, Q, page_size, seq_lens, bad_pages=True, extra_w=3, lo=-3, hi=3):
+    """Tiny paged decode case with integer data.  Some table entries past the
+    visible range, and (optionally) some inside it, are invalid (-1 or past
+    the pool)."""
+    pages_per_req = [max(1, -(-L // (4 * page_size))) for L in seq_lens]
+    num_pages = sum(pages_per_req) + 2
+    max_pages = max(pages_per_req) + 1
+    perm = rng.permutation(num_pages)
+    table = np.full((B, max_pages), -1, dtype=np.int32)
+    at = 0
+    for b, p in enumerate(pages_per_req):
+        table[b, :p] = perm[at:at + p]
+        at += p
+    if bad_pages and B > 1:
+        table[1, 0] = num_pages + 5          # out of range
+        if pages_per_req[1] > 1:
+            table[1, 1] = -1                  # missing
+    q = int_bf16((B, Q, 4, 128), lo, hi, rng)
+    k_cache = int_bf16((num_pages, page_size, 1, 128), lo, hi, rng)
+    W = max(L // 4 for L in seq_lens) + extra_w
+    return q, k_cache, torch.from_numpy(table), torch.tensor(seq_lens, dtype=torch.int32), W
+
+
+def dense_request_keys(k_cache_int, table_row, page_size, num_pages):
+    """The request's keys in logical order, None where the page is invalid."""
+    keys = []
+    for page in table_row:
+        for r in range(page_size):
+            keys.append(k_cache_int[page, r, 0] if 0 <= page < num_pages else None)
+    return keys
+
+
+def brute_decode(q, k_cache, table, seq_lens, W):
+    qi, ki = as_int(q), as_int(k_cache)
+    B, Q = qi.shape[:2]
+    out = np.full((B, Q, W), -np.inf)
+    for b in range(B):
+        L = int(seq_lens[b])
+        keys = dense_request_keys(ki, table[b].tolist(), k_cache.shape[1], k_cache.shape[0])
+        positions = list(range(L))[-Q:] if L >= Q else [L - Q + i for i in range(Q)]
+        for i, p in enumerate(positions):
+            written = keys_written_through(p) if p >= 0 else []
+            for n in written:
+                if n < W and n < len(keys) and keys[n] is not None:
+                    out[b, i, n] = int_score(qi[b, i], keys[n])
+    return out
+
+
+def packed_case(rng, new_tokens, prefixes, lo=-3, hi=3):
+    total = [p + n for p, n in zip(prefixes, new_tokens)]
+    nkeys = [len(keys_written_through(t - 1)) for t in total]
+    T = sum(new_tokens)
+    q = int_bf16((T, 4, 128), lo, hi, rng)
+    k = int_bf16((sum(nkeys), 128), lo, hi, rng)
+    cu = np.concatenate([[0], np.cumsum(new_tokens)]).astype(np.int32)
+    offs = np.concatenate([[0], np.cumsum(nkeys)[:-1]]).astype(np.int32)
+    return q, k, cu, np.array(total, dtype=np.int32), offs, max(nkeys)
+
+
+# ---------------------------------------------------------------- the mask
+
+def pin_visible_blocks_follow_cache_writer(orc):
+    for L in range(0, 41):
+        for p in range(0, L):
+            written = keys_written_through(p)
+            assert written == list(range(len(written)))
+            v = orc.visible_blocks(p, L)
+            assert v == len(written), (p, L, v, len(written))
+        # a padding row (logical position -1) sees nothing
+        assert orc.visible_blocks(-1, L) == 0
+        # positions past the request are capped at the keys the cache holds
+        assert orc.visible_blocks(L + 9, L) == len(keys_written_through(L - 1))
+
+
+def pin_decode_positions_are_last_tokens(orc):
+    for L in range(1, 30):
+        for Q in range(1, min(L, 4) + 1):
+            expect = list(range(L))[-Q:]
+            got = [orc.logical_position(L, Q, i) for i in range(Q)]
+            assert got == expect, (L, Q, got, expect)
+            vis = orc.decode_visible([L], Q)[0].tolist()
+            assert vis == [len(keys_written_through(p)) for p in expect]
+    # fewer tokens than query rows: the leading rows have no position
+    assert orc.decode_visible([2], 4)[0].tolist() == [0, 0, 0, 0]
+
+
+def pin_prefill_flops_match_published_table(orc):
+    rows = 0
+    with open(GOLDEN) as f:
+        for line in f:
+            parts = line.split()
+            if not parts or parts[0] != "prefill":
+                continue
+            S, n = map(int, parts[1].split("x"))
+            prefix = int(parts[2])
+            cu = [i * n for i in range(S + 1)]
+            ks, ke = orc.prefill_intervals(cu, [prefix + n] * S, [0] * S)
+            flop = 2 * 4 * 128 * int((ke.astype(np.int64) - ks).sum())
+            for us, printed in ((float(parts[3]), float(parts[5])),
+                                (float(parts[4]), float(parts[6]))):
+                got = round(flop / us / 1e6, 1)
+                assert got == printed, (parts[1], prefix, us, got, printed)
+            rows += 1
+    assert rows == 12
+
+
+def pin_prefill_intervals_follow_cache_writer(orc):
+    new, pre = [5, 1, 9, 3], [0, 7, 13, 2]
+    cu = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+    total = [a + b for a, b in zip(pre, new)]
+    offs = [0, 11, 30, 50]
+    ks, ke = orc.prefill_intervals(cu, total, offs)
+    t = 0
+    for s in range(4):
+        for i in range(new[s]):
+            p = pre[s] + i
+            assert ks[t] == offs[s]
+            assert ke[t] - ks[t] == len(keys_written_through(p)), (s, i)
+            t += 1
+
+
+# ---------------------------------------------------------------- the score
+
+def pin_decode_exact_bruteforce(orc):
+    rng = np.random.default_rng(1)
+    cases = [(1, 1, 8, [37]), (3, 4, 8, [70, 41, 2]), (2, 2, 16, [130, 75]),
+             (3, 3, 8, [0, 66, 19]), (2, 4, 16, [64, 3])]
+    for B, Q, ps, lens in cases:
+        q, kc, table, sl, W = paged_case(rng, B, Q, ps, lens)
+        got = orc.decode(q, kc, table, sl, W, scale=1.0, threads=2)
+        want = brute_decode(q, kc, table.numpy(), sl.numpy(), W)
+        assert np.array_equal(got, want), (B, Q, ps, lens)
+
+
+def pin_prefill_exact_bruteforce(orc):
+    rng = np.random.default_rng(2)
+    new, pre = [6, 3, 9], [5, 0, 22]
+    q, k, cu, total, offs, Wmax = packed_case(rng, new, pre)
+    ks, ke = orc.prefill_intervals(cu, total, offs)
+    W = Wmax + 2
+    got = orc.prefill(q, k, ks, ke, W, scale=1.0, threads=2)
+    qi, ki = as_int(q), as_int(k)
+    want = np.full((q.shape[0], W), -np.inf)
+    t = 0
+    for s in range(3):
+        for i in range(new[s]):
+            for n in keys_written_through(pre[s] + i):
+                want[t, n] = int_score(qi[t], ki[offs[s] + n])
+            t += 1
+    assert np.array_equal(got, want)
+    # arbitrary intervals, clipped to the key range, column j holding key ks + j
+    T, Nk = q.shape[0], k.shape[0]
+    ks2 = rng.integers(-4, Nk, size=T).astype(np.int32)
+    ke2 = (ks2 + rng.integers(-2, 9, size=T)).astype(np.int32)
+    ke2[0], ks2[1], ke2[1] = Nk + 5, -3, 4
+    got2 = orc.prefill(q, k, ks2, ke2, 12, scale=1.0)
+    for t in range(T):
+        for j in range(12):
+            n = int(ks2[t]) + j
+            ok = max(int(ks2[t]), 0) <= n < min(int(ke2[t]), Nk)
+            want_tj = int_score(qi[t], ki[n]) if ok else -np.inf
+            assert got2[t, j] == want_tj, (t, j)
+
+
+def pin_closed_forms(orc):
+    T = 3
+    q = torch.zeros(T, 4, 128, dtype=torch.bfloat16)
+    k = torch.zeros(4, 128, dtype=torch.bfloat16)
+    q[0, 2, :] = 1.0                       # one head all ones
+    k[0, :] = 1.0                          # key all ones
+    k[1, 17] = 1.0                         # key = e_17
+    q[1] = torch.tensor(np.random.default_rng(3).normal(size=(4, 128)), dtype=torch.bfloat16)
+    q[2] = 1.0
+    k[2, :] = -1.0                         # every dot product negative
+    ks = np.zeros(T, dtype=np.int32)
+    ke = np.full(T, 4, dtype=np.int32)
+    s = orc.prefill(q, k, ks, ke, 4, scale=SCALE)
+    assert abs(s[0, 0] - math.sqrt(128.0)) <= 1e-12
+    want = SCALE * sum(max(float(q[1, h, 17]), 0.0) for h in range(4))
+    assert abs(s[1, 1] - want) <= 1e-15
+    assert s[2, 2] == 0.0
+    assert s[0, 3] == 0.0 and s[1, 3] == 0.0  # zero key
+    assert abs(s[2, 0] - 4 * 128 * SCALE) <= 1e-12
+
+
+def pin_invariants(orc):
+    rng = np.random.default_rng(4)
+    B, Q, ps, lens = 3, 4, 8, [90, 33, 61]
+    q, kc, table, sl, W = paged_case(rng, B, Q, ps, lens, bad_pages=False, lo=-8, hi=8)
+    base = orc.decode(q, kc, table, sl, W)
+    vis = orc.decode_visible(sl, Q)
+    cols = np.arange(W)[None, None, :]
+    unmasked = cols < vis[:, :, None]
+    assert np.all(base[unmasked] >= 0.0)
+    assert np.all(np.isneginf(base[~unmasked]))
+    # zero queries give zeros where unmasked
+    z = orc.decode(torch.zeros_like(q), kc, table, sl, W)
+    assert np.all(z[unmasked] == 0.0) and np.all(np.isneginf(z[~unmasked]))
+    # moving pages to other slots of the pool changes nothing
+    P = kc.shape[0]
+    perm = rng.permutation(P)
+    kc2 = torch.empty_like(kc)
+    kc2[torch.from_numpy(perm)] = kc
+    t2 = table.numpy().copy()
+    t2[t2 >= 0] = perm[t2[t2 >= 0]]
+    assert np.array_equal(orc.decode(q, kc2, torch.from_numpy(t2), sl, W), base)
+    # scaling keys by c > 0 scales scores by c: exactly for powers of two, and
+    # exactly for any c once the 1/sqrt(128) multiplier is left out
+    for c in (2.0, 0.5):
+        sc = orc.decode(q, (kc.float() * c).to(torch.bfloat16), table, sl, W)
+        assert np.array_equal(sc[unmasked], c * base[unmasked])
+    unscaled = orc.decode(q, kc, table, sl, W, scale=1.0)
+    for c in (3.0, 5.0):
+        sc = orc.decode(q, (kc.float() * c).to(torch.bfloat16), table, sl, W, scale=1.0)
+        assert np.array_equal(sc[unmasked], c * unscaled[unmasked])
+
+
+def pin_cross_entry_identities(orc):
+    rng = np.random.default_rng(5)
+    B, Q, ps, lens = 2, 4, 8, [77, 45]
+    q, kc, table, sl, W = paged_case(rng, B, Q, ps, lens, bad_pages=False, lo=-8, hi=8)
+    spec = orc.decode(q, kc, table, sl, W)
+    # spec-decode row i == single-token decode of the request cut after that token
+    for i in range(Q):
+        sl_i = sl - Q + i + 1
+        one = orc.decode(q[:, i:i + 1], kc, table, sl_i, W)
+        assert np.array_equal(one[:, 0], spec[:, i]), i
+    # paged decode == prefill over the request's keys laid out densely
+    vis = orc.decode_visible(sl, Q)
+    for b in range(B):
+        pages = [p for p in table[b].tolist() if p >= 0]
+        dense = torch.cat([kc[p, :, 0, :] for p in pages], dim=0)
+        ks = np.zeros(Q, dtype=np.int32)
+        ke = vis[b].astype(np.int32)
+        pre = orc.prefill(q[b], dense, ks, ke, W)
+        assert np.array_equal(pre, spec[b]), b
+    # the same keys paged with 16 rows per page instead of 8
+    keys = [torch.cat([kc[p, :, 0, :] for p in table[b].tolist() if p >= 0]) for b in range(B)]
+    ps2 = 16
+    pool, t16 = [], np.full((B, 8), -1, dtype=np.int32)
+    for b in range(B):
+        kb = keys[b]
+        pad = (-kb.shape[0]) % ps2
+        kb = torch.cat([kb, torch.zeros(pad, 128, dtype=kb.dtype)])
+        for j in range(kb.shape[0] // ps2):
+            t16[b, j] = len(pool)
+            pool.append(kb[j * ps2:(j + 1) * ps2])
+    kc16 = torch.stack(pool)[:, :, None, :]
+    assert np.array_equal(orc.decode(q, kc16, torch.from_numpy(t16), sl, W), spec)
+    # longer intervals leave earlier columns unchanged
+    Tq = q[0]
+    ks = np.zeros(Q, dtype=np.int32)
+    short = orc.prefill(Tq, keys[0], ks, np.full(Q, 5, dtype=np.int32), 12)
+    longer = orc.prefill(Tq, keys[0], ks, np.full(Q, 12, dtype=np.int32), 12)
+    assert np.array_equal(short[:, :5], longer[:, :5])
+
+
+# ---------------------------------------------------------------- top-k
+
+def pin_topk_against_full_sort(orc):
+    rng = np.random.default_rng(6)
+    rows, width, k = 40, 300, 16
+    s = rng.normal(size=(rows, width))
+    lengths = rng.integers(0, width + 1, size=rows).astype(np.int32)
+    lengths[:4] = [0, 5, 16, width]
+    got = orc.topk(s, lengths, k)
+    for r in range(rows):
+        L = int(lengths[r])
+        order = np.argsort(-s[r, :L], kind="stable")[:k]
+        want = sorted(order.tolist()) + [-1] * (k - min(k, L))
+        assert got[r].tolist() == want, r
+
+
+def pin_topk_ties_and_padding(orc):
+    k = 4
+    s = np.array([
+        [1.0] * 10,                                              # all tied: lowest columns
+        [0.0, -0.0, 0.0, -0.0, 5.0, 0.0, 0.0, 0.0, 0.0, 0.0],    # signed zeros tie
+        [3.0, -np.inf, 2.0, -np.inf, 1.0, 0.0, 0.0, 0.0, 0.0, 0.0],
+        [2.0, 1.0, 3.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0],
+    ])
+    lengths = np.array([10, 10, 4, 2], dtype=np.int32)
+    got = orc.topk(s, lengths, k)
+    assert got[0].tolist() == [0, 1, 2, 3]
+    assert got[1].tolist() == [0, 1, 2, 4]
+    assert got[2].tolist() == [0, 1, 2, 3]
+    assert got[3].tolist() == [0, 1, -1, -1]
+
+
+ALL_PINS = [
+    pin_visible_blocks_follow_cache_writer,
+    pin_decode_positions_are_last_tokens,
+    pin_prefill_flops_match_published_table,
+    pin_prefill_intervals_follow_cache_writer,
+    pin_decode_exact_bruteforce,
+    pin_prefill_exact_bruteforce,
+    pin_closed_forms,
+    pin_invariants,
+    pin_cross_entry_identities,
+    pin_topk_against_full_sort,
+    pin_topk_ties_and_padding,
+]

@@ -261,11 +261,14 @@ void qsa_oracle_prefill_entries(const uint16_t *q, int64_t q_st, int64_t q_sh,
 /* ------------------------------------------------------------- top-k */
 
 /* Per-row top-k (the caller's selection step in the QSA docs' pipeline;
- * widths 512 / 1024 / 2048 in the vLLM PR's top-k discussion).  Among the
- * first lengths[r] columns of row r, take the min(k, lengths[r]) largest
- * scores, ties going to the lower column; write their column indices in
- * ascending order and pad the rest of the k slots with -1.  -0.0 and +0.0
- * compare equal.  The ordering is done by the C library's qsort. */
+ * widths 512 / 1024 / 2048 in the vLLM PR's top-k discussion).  The
+ * candidates of row r are its first lengths[r] columns whose score is not
+ * masked: a -inf (or NaN) score marks a block the row cannot see, and the
+ * selection runs over visible blocks only.  Take the min(k, #candidates)
+ * largest scores, ties going to the lower column; write their column
+ * indices in ascending order and pad the rest of the k slots with -1.
+ * -0.0 and +0.0 compare equal.  The ordering is done by the C library's
+ * qsort. */
 
 typedef struct { double v; int64_t j; } scored_col;
 
@@ -292,14 +295,18 @@ static void topk_rows(void *vctx, int64_t begin, int64_t end) {
     for (int64_t r = begin; r < end; ++r) {
         int64_t len = c->lengths[r] > 0 ? c->lengths[r] : 0;
         int32_t *dst = c->idx + r * c->idx_stride;
-        int64_t take = len < c->k ? len : c->k;
+        int64_t ncand = 0, take = 0;
         if (len > 0) {
             scored_col *cols = (scored_col *)malloc(sizeof(scored_col) * (size_t)len);
             for (int64_t j = 0; j < len; ++j) {
-                cols[j].v = c->scores[r * c->stride + j];
-                cols[j].j = j;
+                double v = c->scores[r * c->stride + j];
+                if (!(v > -INFINITY)) continue;  /* masked block (or NaN) */
+                cols[ncand].v = v;
+                cols[ncand].j = j;
+                ++ncand;
             }
-            qsort(cols, (size_t)len, sizeof(scored_col), by_score_desc_then_col);
+            take = ncand < c->k ? ncand : c->k;
+            qsort(cols, (size_t)ncand, sizeof(scored_col), by_score_desc_then_col);
             for (int64_t s = 0; s < take; ++s) dst[s] = (int32_t)cols[s].j;
             free(cols);
             qsort(dst, (size_t)take, sizeof(int32_t), by_col);

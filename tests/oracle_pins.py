@@ -324,13 +324,15 @@ def pin_topk_against_full_sort(orc):
     rng = np.random.default_rng(6)
     rows, width, k = 40, 300, 16
     s = rng.normal(size=(rows, width))
+    s[rng.random(size=s.shape) < 0.05] = -np.inf
     lengths = rng.integers(0, width + 1, size=rows).astype(np.int32)
     lengths[:4] = [0, 5, 16, width]
     got = orc.topk(s, lengths, k)
     for r in range(rows):
         L = int(lengths[r])
-        order = np.argsort(-s[r, :L], kind="stable")[:k]
-        want = sorted(order.tolist()) + [-1] * (k - min(k, L))
+        cand = np.flatnonzero(np.isfinite(s[r, :L]))
+        order = cand[np.argsort(-s[r, cand], kind="stable")][:k]
+        want = sorted(order.tolist()) + [-1] * (k - len(order))
         assert got[r].tolist() == want, r
 
 
@@ -346,8 +348,11 @@ def pin_topk_ties_and_padding(orc):
     got = orc.topk(s, lengths, k)
     assert got[0].tolist() == [0, 1, 2, 3]
     assert got[1].tolist() == [0, 1, 2, 4]
-    assert got[2].tolist() == [0, 1, 2, 3]
+    assert got[2].tolist() == [0, 2, -1, -1]    # masked blocks are never selected
     assert got[3].tolist() == [0, 1, -1, -1]
+    # NaN is not a candidate either
+    s2 = np.array([[np.nan, 1.0, np.nan, 2.0]])
+    assert orc.topk(s2, np.array([4], dtype=np.int32), 3)[0].tolist() == [1, 3, -1]
 
 
 ALL_PINS = [

@@ -30,6 +30,7 @@ MUTANTS = {
         "int64_t hi = a->ke[t] < a->Nk ? a->ke[t] : a->Nk;", "int64_t hi = a->Nk;"),
     "top-k ties to the higher column": ("return (a->j > b->j) - (a->j < b->j);",
                                         "return (a->j < b->j) - (a->j > b->j);"),
+    "top-k selects masked blocks": ("if (!(v > -INFINITY)) continue;", "if (v != v) continue;"),
     "top-k keeps the smallest": ("if (a->v > b->v) return -1;\n    if (a->v < b->v) return 1;",
                                  "if (a->v < b->v) return -1;\n    if (a->v > b->v) return 1;"),
 }

@@ -1,0 +1,518 @@
+"""Benchmark of the QSA MQA indexer score on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl ours|reference]
+
+One step = one pass of the indexer over one batch of the chosen workload
+(default: 16 decode requests, one query token each, log-normal contexts of
+1,536-43,876 tokens, page size 64).  The K timed steps are captured in one
+CUDA graph and replayed between CUDA events on the launching stream, after W
+untimed warm-up steps; the steps rotate over enough copies of the inputs
+that their total exceeds twice the 126 MB L2, so every step reads HBM.
+
+Throughput accounting follows the vLLM PR "Separate prefill and decode
+paths for QSA indexer" (section "Microbenchmarks"), whose printed numbers
+these formulas reproduce (tests/test_bench_accounting.py):
+  decode bytes  = sum_b [(ctx_b // 4) * 256 + DQL * (ctx_b // 4) * 4] + B * DQL * 1024
+  prefill FLOPs = 2 * 4 * 128 * sum_t visible(t)
+
+Under torchrun each rank runs its own replica of the workload (weak
+scaling: the indexer needs no exchange between GPUs); the step time is the
+maximum over ranks and the value counts the work of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "indexer µs and GB/s (decode) / TFLOP/s (prefill) and % of roofline, 1×B200"
+L2_BYTES = 126 * 1024 * 1024
+PUBLISHED = {  # the vLLM PR's GB300 numbers for the same workload shapes (context only)
+    2: ("GB/s", 1302.0, "vLLM PR microbenchmarks, DQL 1, 16 requests, 1,536/10,240/43,876 tokens, GB300, ps 196"),
+    3: ("GB/s", 3374.0, "vLLM PR microbenchmarks, DQL 4, 16 requests, 3,508/51,200/102,400 tokens, GB300, ps 196"),
+}
+
+
+# ------------------------------------------------------------------ accounting
+
+def decode_bytes(seq_lens, dql: int) -> int:
+    """Algorithmic bytes of one decode step: the visible bf16 keys, the fp32
+    scores of the visible blocks and the bf16 queries."""
+    keys = sum(int(L) // 4 for L in seq_lens)
+    return keys * 256 + dql * keys * 4 + len(seq_lens) * dql * 1024
+
+
+def prefill_flops(ks, ke) -> int:
+    """2 * 4 heads * 128 features per (row, visible key) pair."""
+    return 2 * 4 * 128 * int(np.sum(np.asarray(ke, dtype=np.int64) - np.asarray(ks, dtype=np.int64)))
+
+
+def read_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def read_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    if not os.path.exists(path):
+        return None
+    import hashlib
+    src = os.path.join(ROOT, "sparse_attention_block_qsa_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(src)):
+        with open(os.path.join(src, f), "rb") as fh:
+            h.update(fh.read())
+    sha = h.hexdigest()[:12]
+    for line in open(path):
+        parts = [p.strip() for p in line.strip().strip("|").split("|")]
+        if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload and parts[2] == sha:
+            try:
+                return int(parts[3])
+            except ValueError:
+                return None
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workloads
+
+class DecodeBench:
+    """Decode / spec-decode step: one qsa_mqa_decode launch over one batch."""
+    kernel = "decode_kernel"
+    bound = "hbm"
+
+    def __init__(self, cfg: int, dev: torch.device, seed: int):
+        import sparse_attention_block_qsa_b200 as qsa
+        self.qsa = qsa
+        self.inp = wl.make_config(cfg, seed=seed)
+        d = self.inp
+        self.name = d.name
+        self.units = decode_bytes(d.seq_lens.tolist(), d.Q)        # algorithmic bytes per step
+        per_copy = (d.q.numel() + d.k_cache.numel()) * 2 + d.B * d.Q * d.W * 4
+        self.copies = max(2, math.ceil(2 * L2_BYTES / per_copy))
+        self.dev = dev
+        self.bufs = []
+        for _ in range(self.copies):
+            self.bufs.append((d.q.to(dev), d.k_cache.to(dev), d.page_table.to(dev), d.seq_lens.to(dev),
+                              torch.empty((d.B, d.Q, d.W), dtype=torch.float32, device=dev)))
+        self.launches_per_step = 1
+        self.h2d = (d.q.numel() + d.k_cache.numel()) * 2 + (d.page_table.numel() + d.seq_lens.numel()) * 4
+        self.d2h = d.B * d.Q * d.W * 4
+        self.config = {"workload": d.name, "requests": d.B, "query_tokens": d.Q, "page_size": d.page_size,
+                       "context_tokens": d.meta["context_tokens"], "W": d.W, "input_copies": self.copies,
+                       "l2": f"steps rotate over {self.copies} input copies "
+                             f"({self.copies * per_copy / 2**20:.0f} MiB > 2x L2)"}
+
+    def step(self, i: int):
+        q, kc, pt, sl, out = self.bufs[i % self.copies]
+        self.qsa.mqa_decode(q, kc, pt, sl, self.inp.W, out=out)
+
+    def throughput(self, seconds_per_step: float) -> float:
+        return self.units / seconds_per_step / 1e9   # GB/s
+
+    unit = "GB/s"
+
+    def e2e_setup(self):
+        d = self.inp
+        self.host = [t.pin_memory() for t in (d.q, d.k_cache, d.page_table, d.seq_lens)]
+        self.host_out = torch.empty((d.B, d.Q, d.W), dtype=torch.float32).pin_memory()
+
+    def e2e_step(self, i: int):
+        q, kc, pt, sl, out = self.bufs[i % self.copies]
+        for dst, src in zip((q, kc, pt, sl), self.host):
+            dst.copy_(src, non_blocking=True)
+        self.qsa.mqa_decode(q, kc, pt, sl, self.inp.W, out=out)
+        self.host_out.copy_(out, non_blocking=True)
+
+    def oracle_step(self, threads: int = 0):
+        import oracle
+        d = self.inp
+        oracle.decode(d.q, d.k_cache, d.page_table, d.seq_lens, d.W, threads=threads)
+
+    def oracle_sample(self):
+        return 1.0, "one full step (every score of the batch)"
+
+
+class PrefillBench:
+    """Prefill step: qsa_mqa_prefill (configuration 4) or the fused prefill
+    + top-512 (configuration 5) over one packed batch."""
+    kernel = "prefill_kernel"
+    bound = "tensor"
+    unit = "TFLOP/s"
+
+    def __init__(self, cfg: int, dev: torch.device, seed: int):
+        import sparse_attention_block_qsa_b200 as qsa
+        self.qsa = qsa
+        self.cfg = cfg
+        self.inp = p = wl.make_config(cfg, seed=seed)
+        self.name = p.name
+        self.dev = dev
+        self.q, self.k = p.q.to(dev), p.k.to(dev)
+        self.cu, self.sl, self.ko = p.cu_seqlens_q.to(dev), p.seq_lens.to(dev), p.key_offsets.to(dev)
+        self.ks, self.ke = qsa.prefill_intervals(self.cu, self.sl, self.ko, p.T)
+        ks_h, ke_h = self.ks.cpu().numpy(), self.ke.cpu().numpy()
+        self.units = prefill_flops(ks_h, ke_h)
+        self.topk = cfg == 5
+        self.out = torch.empty((p.T, p.W), dtype=torch.float32, device=dev)
+        if self.topk:
+            self.idx = torch.empty((p.T, wl.TOPK_K), dtype=torch.int32, device=dev)
+        self.copies = 1
+        self.launches_per_step = 2 if self.topk else 1
+        out_bytes = p.T * p.W * 4
+        self.h2d = (p.q.numel() + p.k.numel()) * 2 + (p.cu_seqlens_q.numel() + 2 * p.seq_lens.numel()) * 4
+        self.d2h = p.T * wl.TOPK_K * 4 if self.topk else out_bytes
+        self.config = {"workload": p.name, "sequences": len(p.meta["new_tokens"]),
+                       "new_tokens": p.meta["new_tokens"], "prefix_tokens": p.meta["prefix_tokens"],
+                       "keys": p.Nk, "W": p.W, "flop_per_step": self.units,
+                       "l2": f"each step writes {out_bytes / 2**20:.0f} MiB of scores (> L2)"}
+        if self.topk:
+            self.config["topk"] = wl.TOPK_K
+
+    def step(self, i: int, mid_event=None):
+        p = self.inp
+        self.qsa.mqa_prefill(self.q, self.k, self.ks, self.ke, p.W, out=self.out)
+        if self.topk:
+            if mid_event is not None:
+                mid_event.record()
+            self.qsa.topk(self.out, wl.TOPK_K, idx=self.idx)
+
+    def throughput(self, seconds_per_step: float) -> float:
+        return self.units / seconds_per_step / 1e12
+
+    def e2e_setup(self):
+        p = self.inp
+        self.host = [t.pin_memory() for t in (p.q, p.k, p.cu_seqlens_q, p.seq_lens, p.key_offsets)]
+        shape = (p.T, wl.TOPK_K) if self.topk else (p.T, p.W)
+        self.host_out = torch.empty(shape, dtype=torch.int32 if self.topk else torch.float32).pin_memory()
+
+    def e2e_step(self, i: int):
+        p = self.inp
+        for dst, src in zip((self.q, self.k, self.cu, self.sl, self.ko), self.host):
+            dst.copy_(src, non_blocking=True)
+        self.qsa.prefill_intervals(self.cu, self.sl, self.ko, p.T, ks=self.ks, ke=self.ke)
+        self.step(i)
+        self.host_out.copy_(self.idx if self.topk else self.out, non_blocking=True)
+
+    def oracle_sample(self):
+        return 64 / self.inp.T, "64 query rows of the batch, every column (scaled to the full batch)"
+
+    def oracle_step(self, threads: int = 0):
+        import oracle
+        p = self.inp
+        ks, ke = oracle.prefill_intervals(p.cu_seqlens_q, p.seq_lens, p.key_offsets)
+        rows = slice(0, 64)
+        s = oracle.prefill(p.q[rows], p.k, ks[rows], ke[rows], p.W, threads=threads)
+        if self.topk:
+            oracle.topk(s, np.full(s.shape[0], p.W, dtype=np.int32), wl.TOPK_K, threads=threads)
+
+
+def make_bench(cfg: int, dev, seed: int):
+    return DecodeBench(cfg, dev, seed) if cfg in (1, 2, 3) else PrefillBench(cfg, dev, seed)
+
+
+# ------------------------------------------------------------------ timing
+
+def sync_all(world: int):
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_graph(b, steps: int, world: int, soak_s: float = 0.0, sampler: ClockSampler | None = None):
+    """Capture `steps` steps in one graph; return (seconds per step, seconds
+    per step of the dominant kernel, clocks)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for i in range(steps):
+                b.step(i)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.start()
+    t_end = time.time() + soak_s
+    while time.time() < t_end:
+        g.replay()
+        torch.cuda.synchronize()
+    sync_all(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    g.replay()
+    end.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler is not None else None
+    sync_all(world)
+    elapsed = start.elapsed_time(end) / 1e3
+    del g
+    return elapsed / steps, clocks
+
+
+def time_kernel_split(b, reps: int = 10):
+    """For a two-kernel step: per-kernel seconds (prefill, top-k), events
+    around each kernel on the launching stream."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, m, e in ev:
+        a.record()
+        b.step(0, mid_event=m)
+        e.record()
+    torch.cuda.synchronize()
+    pre = statistics.median(a.elapsed_time(m) for a, m, _ in ev) / 1e3
+    top = statistics.median(m.elapsed_time(e) for _, m, e in ev) / 1e3
+    return pre, top
+
+
+def time_e2e(b, steps: int, warmup: int, world: int):
+    b.e2e_setup()
+    for i in range(warmup):
+        b.e2e_step(i)
+    sync_all(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        b.e2e_step(i)
+    end.record()
+    torch.cuda.synchronize()
+    sync_all(world)
+    return start.elapsed_time(end) / 1e3 / steps
+
+
+def cpu_baseline(b, budget_s: float = 10.0) -> dict:
+    import oracle
+    threads = oracle.default_threads()
+    frac, what = b.oracle_sample()
+    b.oracle_step(threads)          # builds / loads the oracle, warms caches
+    n, t0 = 0, time.perf_counter()
+    while True:
+        b.oracle_step(threads)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s or n >= 50:
+            break
+    per_sample = (time.perf_counter() - t0) / n
+    per_step = per_sample / frac
+    return {"value": b.throughput(per_step), "unit": b.unit, "cores": threads, "kind": "oracle",
+            "sample": f"{what}; {n} repetitions, {per_sample:.3f} s each, fp64 C oracle on {threads} host threads",
+            "seconds_per_step": per_step}
+
+
+# ------------------------------------------------------------------ main
+
+def run_reference(args, rank: int, world: int):
+    """The oracle as the reference arm, timed on the host cores."""
+    if rank != 0:
+        return
+    dev = torch.device("cpu")
+    import oracle
+    inp_bench = _HostOnly(args.config)
+    threads = oracle.default_threads()
+    frac, what = inp_bench.oracle_sample()
+    for _ in range(args.warmup):
+        inp_bench.oracle_step(threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        inp_bench.oracle_step(threads)
+    per_sample = (time.perf_counter() - t0) / args.steps
+    per_step = per_sample / frac
+    value = inp_bench.throughput(per_step)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": inp_bench.unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": inp_bench.config,
+            "cpu_baseline": {"value": value, "unit": inp_bench.unit, "cores": threads, "kind": "oracle",
+                             "sample": f"{what}; fp64 C oracle on {threads} host threads"},
+            "e2e": {"value": value, "unit": inp_bench.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+class _HostOnly:
+    """Inputs and accounting of a workload without any GPU state."""
+
+    def __init__(self, cfg: int):
+        self.cfg = cfg
+        self.inp = wl.make_config(cfg)
+        if cfg in (1, 2, 3):
+            d = self.inp
+            self.units = decode_bytes(d.seq_lens.tolist(), d.Q)
+            self.unit = "GB/s"
+            self.config = {"workload": d.name, "requests": d.B, "query_tokens": d.Q, "page_size": d.page_size,
+                           "W": d.W}
+        else:
+            import oracle
+            p = self.inp
+            ks, ke = oracle.prefill_intervals(p.cu_seqlens_q, p.seq_lens, p.key_offsets)
+            self.units = prefill_flops(ks, ke)
+            self.unit = "TFLOP/s"
+            self.config = {"workload": p.name, "keys": p.Nk, "W": p.W}
+
+    def throughput(self, s):
+        return self.units / s / (1e9 if self.unit == "GB/s" else 1e12)
+
+    def oracle_sample(self):
+        if self.cfg in (1, 2, 3):
+            return 1.0, "one full step (every score of the batch)"
+        return 64 / self.inp.T, "64 query rows of the batch, every column (scaled to the full batch)"
+
+    def oracle_step(self, threads):
+        if self.cfg in (1, 2, 3):
+            DecodeBench.oracle_step(self, threads)
+        else:
+            PrefillBench.oracle_step(self, threads)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--soak", type=float, default=1.5, help="seconds of load before the timed region")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+
+    b = make_bench(args.config, dev, seed=rank)
+    for i in range(args.warmup):
+        b.step(i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if rank == 0 else None
+    per_step, clocks = time_graph(b, args.steps, world, soak_s=args.soak, sampler=sampler)
+    per_step = max_over_ranks(per_step, world)
+    kernel_s = per_step
+    split = None
+    if b.launches_per_step == 2:
+        pre, top = time_kernel_split(b)
+        kernel_s = pre
+        split = {"prefill_us": pre * 1e6, "topk_us": top * 1e6}
+    e2e_s = max_over_ranks(time_e2e(b, args.steps, 3, world), world)
+    from sparse_attention_block_qsa_b200 import device_error
+    dev_err = device_error()
+
+    if rank == 0:
+        peaks = read_peaks()
+        value = b.throughput(per_step) * world
+        if b.bound == "hbm":
+            achieved = b.units / kernel_s / 1e9
+            peak, unit = peaks["hbm_gbs"], "GB/s"
+        else:
+            achieved = b.units / kernel_s / 1e12
+            peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+        roofline = {"bound": b.bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                    "traffic": read_traffic(b.kernel, b.name), "kernel": b.kernel,
+                    "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst figure)"
+                    if peaks["source"] == "measured" else "fallback"}
+        pub = PUBLISHED.get(args.config)
+        cfg = dict(b.config)
+        if pub:
+            cfg["published_reference"] = pub[2]
+        line = {"metric": METRIC, "value": value, "unit": b.unit, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": per_step * 1e3, "us_per_step": per_step * 1e6,
+                "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": (value / pub[1]) if pub and pub[0] == b.unit else None,
+                "dtype": "bf16", "data": "synthetic", "config": cfg,
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "roofline": roofline,
+                "e2e": {"value": b.throughput(e2e_s) * world, "unit": b.unit, "h2d_bytes_per_step": b.h2d,
+                        "d2h_bytes_per_step": b.d2h, "ms_per_step": e2e_s * 1e3},
+                "gpu_launches": args.steps * b.launches_per_step,
+                "clocks": clocks, "device_error": dev_err}
+        if split:
+            line["kernels"] = split
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline(b)
+            cb.pop("seconds_per_step", None)
+            line["cpu_baseline"] = cb
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+/*
+ * qsa.h - C ABI of the QSA (Qwen Sparse Attention) MQA indexer score for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The indexer scores compressed 4-token key blocks for every query token:
+ *
+ *     score[t, n] = scale * sum_{h<4} max(0, q[t, h, :] . k[n, :])
+ *
+ * with 4 query heads of dimension 128 sharing one compressed key head of
+ * dimension 128, and scale = 1/sqrt(128) by default (QSA docs, MATE, section
+ * "MQA score": "Scores sum the four head-wise ReLU dot products, scaled by
+ * 1/sqrt(128)"; "scale is a multiplier").  Blocks that are not yet complete
+ * or lie in the future are masked to -inf.  A query token at logical
+ * position pos = seq_len - query_len + i (vLLM qsa_cache.py,
+ * "_logical_positions") sees the compressed keys
+ *
+ *     n < visible = max(0, min((pos + 1) / 4, seq_len / 4))   (floor division)
+ *
+ * (vLLM qsa_cache.py, metadata kernel, "visible_blocks"; the vLLM PR
+ * "Separate prefill and decode paths for QSA indexer", section "Main changes",
+ * names the same quantity).
+ *
+ * Conventions shared by every call:
+ *  - Pointers named q, k, k_cache, page_table, seq_lens, ks, ke, lengths,
+ *    scores, out, idx, workspace are DEVICE pointers owned by the caller.
+ *    The library allocates nothing, never synchronises the stream and never
+ *    reads device memory from the host; every call is asynchronous on
+ *    `stream` (a cudaStream_t; NULL means the legacy default stream).
+ *  - bf16 tensors are passed as raw pointers with strides in ELEMENTS; the
+ *    feature (last) stride is always 1.
+ *  - Host-side validation runs before any launch.  On a non-OK status nothing
+ *    was launched and qsa_last_error_detail() describes the problem.
+ *  - Kernels never trap.  A device-side wait that runs out of time sets a bit
+ *    in the library's device error word (qsa_device_error) and the kernel
+ *    returns early; the output is then incomplete.
+ */
+#ifndef QSA_H_
+#define QSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qsa_status {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1, /* a size, count, pointer or value is out of range */
+  QSA_ERR_ALIGNMENT = 2,   /* a base address or stride breaks the layout rules */
+  QSA_ERR_UNSUPPORTED = 3, /* a configuration this build does not implement */
+  QSA_ERR_WORKSPACE = 4,   /* the workspace is too small */
+  QSA_ERR_CUDA = 5         /* a CUDA runtime/driver call or a launch failed */
+} qsa_status_t;
+
+/* Bits of the device error word. */
+#define QSA_DEVERR_WAIT_TIMEOUT 0x1u /* an mbarrier wait ran out of time */
+#define QSA_DEVERR_SELECT 0x2u       /* top-k threshold search did not converge */
+
+/* Static text for a status code. */
+const char* qsa_status_string(qsa_status_t status);
+
+/* Detail of the last non-OK status returned on the calling host thread
+ * (thread-local; empty string if none). */
+const char* qsa_last_error_detail(void);
+
+/* Reads the device error word of the current device into *bits and clears
+ * it.  This call synchronises the device (it is for tests and diagnostics,
+ * never for the hot path). */
+qsa_status_t qsa_device_error(uint32_t* bits);
+
+/*
+ * qsa_mqa_decode - decode and speculative-decode scores over a paged
+ * compressed key cache.
+ *
+ * Defined by the QSA docs (MATE), section "MQA score" ("qsa_mqa_decode takes
+ * paged compressed keys [pages, page_size, 1, dim], a page table and
+ * compressed context lengths"; the context length is passed here in TOKENS
+ * so that each of the Q query tokens gets its own causal visible count), with
+ * the page addressing of vLLM qsa_cache.py, "_logical_to_physical_qsa_slots".
+ *
+ *   q          bf16 [B, Q, 4, 128]; element (b, i, h, c) at
+ *              q + b*q_stride_b + i*q_stride_t + h*q_stride_h + c.
+ *              Strides are non-negative multiples of 8; a stride of 0
+ *              broadcasts that axis.  16-byte aligned.
+ *   k_cache    bf16 [num_pages, page_size, 1, 128]; row r of page p at
+ *              k_cache + p*k_page_stride + r*k_row_stride.  16-byte aligned,
+ *              both strides multiples of 8, k_row_stride >= 128.
+ *   page_size  8, 16, 32 or 64.
+ *   page_table int32 [B, max_pages], row stride pt_stride (>= max_pages).
+ *              Key n of request b lives in page page_table[b, n / page_size]
+ *              at row n % page_size.  Entries may be -1; an entry that is
+ *              negative or >= num_pages (or a block past max_pages) masks the
+ *              keys it would hold to -inf.
+ *   seq_lens   int32 [B]: tokens of request b, its Q query tokens included.
+ *              Query row i sits at logical position seq_lens[b] - Q + i.
+ *   Q          query tokens per request, 1..4 (4 = three speculative tokens).
+ *   scale      score multiplier (1/sqrt(128) for the QSA indexer); finite.
+ *   out        fp32 [B, Q, W]; element (b, i, n) at
+ *              out + b*out_stride_b + i*out_stride_t + n.
+ *              out[b, i, n] = score for n < visible(b, i), else -inf, for
+ *              every n < W (columns past the visible keys are filled with
+ *              -inf).  W >= max visible is the caller's choice; keys at
+ *              n >= W are not scored.  out must not overlap any input.
+ */
+qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
+                            const void* k_cache, int64_t num_pages, int32_t page_size, int64_t k_page_stride,
+                            int64_t k_row_stride, const int32_t* page_table, int64_t pt_stride,
+                            int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t Q, float scale,
+                            float* out, int64_t out_stride_b, int64_t out_stride_t, int32_t W, void* stream);
+
+/*
+ * qsa_mqa_prefill - prefill scores of packed query rows against shared keys
+ * with one key interval per row.
+ *
+ * Defined by the QSA docs (MATE), section "MQA score" ("qsa_mqa_prefill takes
+ * packed queries, shared keys and per-row key intervals").  Column j of row t
+ * holds key ks[t] + j (request-local block index, the frame in which the
+ * docs' "Core Attention" section consumes selected blocks).
+ *
+ *   q        bf16 [T, 4, 128]; element (t, h, c) at q + t*q_stride_t +
+ *            h*q_stride_h + c.  16-byte aligned, strides positive multiples
+ *            of 8 (q_stride_t is free when T == 1).
+ *   k        bf16 [Nk, 128], row stride k_stride (multiple of 8, >= 128).
+ *            16-byte aligned.
+ *   ks, ke   int32 [T]: row t sees keys n with max(ks[t], 0) <= n <
+ *            min(ke[t], Nk); an empty interval gives a row of -inf.
+ *   out      fp32 [T, W], row stride out_stride (>= W when T > 1):
+ *            out[t, j] = score(t, ks[t] + j) if that key is in the row's
+ *            interval, else -inf, for every j < W.  Must not overlap inputs.
+ *   T        rows, 0 <= T <= 16,777,216.
+ */
+qsa_status_t qsa_mqa_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
+                             int64_t k_stride, int64_t Nk, const int32_t* ks, const int32_t* ke, int64_t T,
+                             float scale, float* out, int64_t out_stride, int32_t W, void* stream);
+
+/*
+ * qsa_prefill_intervals - per-row key intervals of a packed prefill batch,
+ * computed on the device (one thread per row).
+ *
+ * Sequence s owns query rows cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1, has
+ * seq_lens[s] tokens in all (cached prefix plus its query rows) and its
+ * compressed keys start at key_offsets[s] in the packed key array.  Row
+ * t = cu_seqlens_q[s] + i gets ks[t] = key_offsets[s] and
+ * ke[t] = key_offsets[s] + visible(pos), pos = seq_lens[s] - qlen_s + i
+ * (vLLM qsa_cache.py, "_logical_positions" and "visible_blocks").
+ *
+ *   cu_seqlens_q int32 [S + 1], non-decreasing, cu_seqlens_q[0] == 0,
+ *                cu_seqlens_q[S] == T.  seq_lens, key_offsets int32 [S].
+ *   ks, ke       int32 [T] outputs.
+ */
+qsa_status_t qsa_prefill_intervals(const int32_t* cu_seqlens_q, const int32_t* seq_lens,
+                                   const int32_t* key_offsets, int32_t S, int64_t T, int32_t* ks, int32_t* ke,
+                                   void* stream);
+
+/*
+ * qsa_topk - per-row top-k block selection over score rows.
+ *
+ * The selection step between the indexer and core attention (QSA docs,
+ * MATE: the caller keeps the top-scoring blocks; "Core Attention": block
+ * hint widths from 1 to 512; the vLLM PR's review thread uses top-k widths
+ * 512, 1024 and 2048).  Among columns j < len(r) of row r whose score is not
+ * -inf (masked blocks are never selected) the k largest are kept, ties going
+ * to the lower column; their column indices are written in ascending order
+ * to idx[r, 0..], and the remaining slots are -1.  -0.0 and +0.0 compare
+ * equal.  NaN scores are never selected.
+ *
+ *   scores   fp32 [rows, W], row stride score_stride (>= W when rows > 1),
+ *            4-byte aligned.
+ *   lengths  int32 [rows] or NULL: len(r) = min(max(lengths[r], 0), W);
+ *            with NULL, len(r) = W.
+ *   k        1..2048.
+ *   idx      int32 [rows, k], row stride idx_stride (>= k when rows > 1).
+ *   W        1..65536.
+ */
+qsa_status_t qsa_topk(const float* scores, int64_t score_stride, const int32_t* lengths, int64_t rows,
+                      int32_t W, int32_t k, int32_t* idx, int64_t idx_stride, void* stream);
+
+/*
+ * qsa_mqa_prefill_topk - prefill scores followed by per-row top-k, without
+ * materialising more than one workspace of scores at a time.
+ *
+ * Rows are processed in chunks whose scores fit in the workspace (the vLLM
+ * PR, "Main changes": prefill logits are bounded by a workspace limit and
+ * processed chunk by chunk); each chunk runs qsa_mqa_prefill into the
+ * workspace (row stride W) and then qsa_topk over it.  Arguments as for the
+ * two calls; the result is idx only.  The workspace must hold at least
+ * min(T, 128) rows of W floats and be 16-byte aligned;
+ * qsa_prefill_topk_workspace_size gives the size that needs a single chunk.
+ * A workspace of a few tens of MB lets the chunk's scores stay in the
+ * B200's 126 MB L2 between the two kernels.
+ */
+qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
+                                  int64_t k_stride, int64_t Nk, const int32_t* ks, const int32_t* ke, int64_t T,
+                                  float scale, int32_t W, int32_t topk_k, int32_t* idx, int64_t idx_stride,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+size_t qsa_prefill_topk_workspace_size(int64_t T, int32_t W);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H_ */

@@ -1,0 +1,47 @@
+"""Build ``libqsa.so`` (the C-ABI library) in-tree with nvcc for sm_100a.
+
+    python -m sparse_attention_block_qsa_b200.build [--force] [--verbose]
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libqsa.so")
+SOURCES = [os.path.join(CSRC, f) for f in ("qsa_lib.cu",)]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "decode.cuh", "prefill.cuh", "topk.cuh")] + [
+    os.path.join(INCLUDE, "qsa.h")]
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+
+def nvcc_command(out: str, verbose: bool = False) -> list[str]:
+    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
+           "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC, *SOURCES, "-o", out]
+    if verbose:
+        cmd += ["-Xptxas", "-v"]
+    return cmd
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    return all(os.path.getmtime(d) <= t for d in DEPS)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and up_to_date():
+        return LIB
+    tmp = LIB + f".tmp{os.getpid()}"
+    subprocess.run(nvcc_command(tmp, verbose), check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))

@@ -1,0 +1,504 @@
+// C ABI of the QSA MQA indexer score (declared in include/qsa.h): host-side
+// validation, TMA tensor-map encoding and kernel launches.  One translation
+// unit, so the kernels and the device error word share one module.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "qsa.h"
+#include "decode.cuh"
+#include "prefill.cuh"
+#include "topk.cuh"
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+qsa_status_t fail(qsa_status_t s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+qsa_status_t ok() {
+  g_detail[0] = '\0';
+  return QSA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// [begin, end) byte range touched by a strided 3-D view (non-negative strides).
+struct Range {
+  uintptr_t lo, hi;
+};
+
+Range span(const void* base, int64_t elem, int64_t n0, int64_t s0, int64_t n1, int64_t s1, int64_t n2, int64_t s2,
+           int64_t inner) {
+  uintptr_t b = reinterpret_cast<uintptr_t>(base);
+  int64_t last = (n0 > 0 ? (n0 - 1) * s0 : 0) + (n1 > 0 ? (n1 - 1) * s1 : 0) + (n2 > 0 ? (n2 - 1) * s2 : 0);
+  return Range{b, b + static_cast<uintptr_t>((last + inner) * elem)};
+}
+
+bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+// ---------------------------------------------------------------- driver entry
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+qsa_status_t encode_bf16_map(CUtensorMap* map, int rank, void* base, const cuuint64_t* dims,
+                             const cuuint64_t* strides_bytes, const cuuint32_t* box, const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides_bytes, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QSA_ERR_ALIGNMENT, "tensor map for %s rejected by the driver (CUresult %d)", what, (int)r);
+  return QSA_OK;
+}
+
+// ---------------------------------------------------------------- device info
+struct DeviceInfo {
+  int sms = 0;
+  bool attrs_set = false;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+qsa_status_t device_info(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(QSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.attrs_set) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+      return fail(QSA_ERR_UNSUPPORTED, "this library is built for sm_100a (B200); device %d is sm_%d%d", dev, major,
+                  minor);
+    e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    struct {
+      const void* fn;
+      size_t bytes;
+    } kernels[] = {
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel), qsa::prefill::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::topk::topk_kernel<true>),
+         sizeof(qsa::topk::Smem) + 4 * (size_t)qsa::topk::MAX_CACHED_W},
+        {reinterpret_cast<const void*>(qsa::topk::topk_kernel<false>), sizeof(qsa::topk::Smem)},
+    };
+    for (auto& k : kernels) {
+      e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k.bytes);
+      if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    }
+    d.attrs_set = true;
+  }
+  *sms = d.sms;
+  return QSA_OK;
+}
+
+qsa_status_t launch_status(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+// ---------------------------------------------------------------- intervals
+__global__ void prefill_intervals_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ seq_lens,
+                                         const int32_t* __restrict__ key_offsets, int32_t S, int64_t T,
+                                         int32_t* __restrict__ ks, int32_t* __restrict__ ke) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  int lo = 0, hi = S - 1;  // last sequence whose first row is <= t
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)__ldg(cu + mid) <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  const int32_t first = __ldg(cu + lo);
+  const int32_t qlen = __ldg(cu + lo + 1) - first;
+  const int32_t L = __ldg(seq_lens + lo);
+  const int32_t pos = L - qlen + (int32_t)(t - first);  // logical position of the row
+  const int32_t vis = max(0, min((pos + 1) >> 2, L >> 2));
+  const int32_t off = __ldg(key_offsets + lo);
+  ks[t] = off;
+  ke[t] = off + vis;
+}
+
+// ---------------------------------------------------------------- prefill core
+struct PrefillArgs {
+  const void* q;
+  int64_t q_stride_t, q_stride_h;
+  const void* k;
+  int64_t k_stride, Nk;
+  const int32_t* ks;
+  const int32_t* ke;
+  int64_t T;
+  float scale;
+  float* out;
+  int64_t out_stride;
+  int32_t W;
+};
+
+qsa_status_t validate_prefill(const PrefillArgs& a) {
+  if (a.T < 0 || a.Nk < 0 || a.W < 0) return fail(QSA_ERR_INVALID_ARG, "T, Nk and W must be non-negative");
+  if (a.T > INT32_MAX) return fail(QSA_ERR_UNSUPPORTED, "T = %lld rows exceeds 2^31 - 1", (long long)a.T);
+  if (a.Nk > INT32_MAX) return fail(QSA_ERR_UNSUPPORTED, "Nk = %lld keys exceeds 2^31 - 1", (long long)a.Nk);
+  if (!std::isfinite(a.scale)) return fail(QSA_ERR_INVALID_ARG, "scale must be finite");
+  if (a.T == 0 || a.W == 0) return QSA_OK;
+  if (!a.q || !a.ks || !a.ke || !a.out || (a.Nk > 0 && !a.k))
+    return fail(QSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(a.q, 16) || (a.Nk > 0 && !aligned(a.k, 16)))
+    return fail(QSA_ERR_ALIGNMENT, "q and k must start on a 16-byte boundary");
+  if (!aligned(a.out, 4) || !aligned(a.ks, 4) || !aligned(a.ke, 4))
+    return fail(QSA_ERR_ALIGNMENT, "out, ks and ke must be 4-byte aligned");
+  if (a.q_stride_h <= 0 || a.q_stride_h % 8 != 0)
+    return fail(QSA_ERR_ALIGNMENT, "q_stride_h = %lld must be a positive multiple of 8", (long long)a.q_stride_h);
+  if (a.T > 1 && (a.q_stride_t <= 0 || a.q_stride_t % 8 != 0))
+    return fail(QSA_ERR_ALIGNMENT, "q_stride_t = %lld must be a positive multiple of 8", (long long)a.q_stride_t);
+  if (a.Nk > 1 && (a.k_stride < 128 || a.k_stride % 8 != 0))
+    return fail(QSA_ERR_ALIGNMENT, "k_stride = %lld must be a multiple of 8 and >= 128", (long long)a.k_stride);
+  if (a.T > 1 && a.out_stride < a.W)
+    return fail(QSA_ERR_INVALID_ARG, "out_stride = %lld is below W = %d", (long long)a.out_stride, a.W);
+  const Range ro = span(a.out, 4, a.T, a.out_stride, 1, 0, 1, 0, a.W);
+  const Range rq = span(a.q, 2, a.T, a.q_stride_t, 4, a.q_stride_h, 1, 0, 128);
+  const Range rks = span(a.ks, 4, a.T, 1, 1, 0, 1, 0, 1), rke = span(a.ke, 4, a.T, 1, 1, 0, 1, 0, 1);
+  if (overlaps(ro, rq) || overlaps(ro, rks) || overlaps(ro, rke) ||
+      (a.Nk > 0 && overlaps(ro, span(a.k, 2, a.Nk, a.k_stride, 1, 0, 1, 0, 128))))
+    return fail(QSA_ERR_INVALID_ARG, "out overlaps an input");
+  return QSA_OK;
+}
+
+qsa_status_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
+  int sms = 0;
+  qsa_status_t st = device_info(&sms);
+  if (st != QSA_OK) return st;
+  CUtensorMap tm_q, tm_k;
+  memset(&tm_k, 0, sizeof tm_k);
+  {
+    const int64_t st_t = a.T > 1 ? a.q_stride_t : 4 * a.q_stride_h;
+    cuuint64_t dims[3] = {128, 4, (cuuint64_t)a.T};
+    cuuint64_t strides[2] = {(cuuint64_t)a.q_stride_h * 2, (cuuint64_t)st_t * 2};
+    cuuint32_t box[3] = {64, 4, (cuuint32_t)qsa::prefill::BT};
+    st = encode_bf16_map(&tm_q, 3, const_cast<void*>(a.q), dims, strides, box, "q");
+    if (st != QSA_OK) return st;
+  }
+  if (a.Nk > 0) {
+    cuuint64_t dims[2] = {128, (cuuint64_t)a.Nk};
+    cuuint64_t strides[1] = {(cuuint64_t)(a.Nk > 1 ? a.k_stride : 128) * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)qsa::prefill::BM};
+    st = encode_bf16_map(&tm_k, 2, const_cast<void*>(a.k), dims, strides, box, "k");
+    if (st != QSA_OK) return st;
+  }
+  for (int64_t r0 = 0; r0 < a.T; r0 += qsa::prefill::MAX_ROWS_PER_LAUNCH) {
+    qsa::prefill::Params p;
+    p.ks = a.ks + r0;
+    p.ke = a.ke + r0;
+    p.q_row0 = (int32_t)r0;
+    p.T = std::min<int64_t>(a.T - r0, qsa::prefill::MAX_ROWS_PER_LAUNCH);
+    p.Nk = a.Nk;
+    p.scale = a.scale;
+    p.out = a.out + r0 * a.out_stride;
+    p.out_stride = a.out_stride;
+    p.W = a.W;
+    qsa::prefill::prefill_kernel<<<sms, qsa::prefill::NUM_THREADS, qsa::prefill::SMEM_BYTES, stream>>>(tm_q, tm_k,
+                                                                                                      p);
+    st = launch_status("prefill kernel");
+    if (st != QSA_OK) return st;
+  }
+  return ok();
+}
+
+// ---------------------------------------------------------------- top-k core
+struct TopkArgs {
+  const float* scores;
+  int64_t score_stride;
+  const int32_t* lengths;
+  int64_t rows;
+  int32_t W, k;
+  int32_t* idx;
+  int64_t idx_stride;
+};
+
+qsa_status_t validate_topk(const TopkArgs& a) {
+  if (a.rows < 0) return fail(QSA_ERR_INVALID_ARG, "rows must be non-negative");
+  if (a.rows > INT32_MAX) return fail(QSA_ERR_UNSUPPORTED, "rows = %lld exceeds 2^31 - 1", (long long)a.rows);
+  if (a.k < 1 || a.k > 2048) return fail(QSA_ERR_UNSUPPORTED, "k = %d must be in [1, 2048]", a.k);
+  if (a.W < 1 || a.W > 65536) return fail(QSA_ERR_UNSUPPORTED, "W = %d must be in [1, 65536]", a.W);
+  if (a.rows == 0) return QSA_OK;
+  if (!a.scores || !a.idx) return fail(QSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(a.scores, 4) || !aligned(a.idx, 4) || (a.lengths && !aligned(a.lengths, 4)))
+    return fail(QSA_ERR_ALIGNMENT, "scores, lengths and idx must be 4-byte aligned");
+  if (a.rows > 1 && a.score_stride < a.W)
+    return fail(QSA_ERR_INVALID_ARG, "score_stride = %lld is below W = %d", (long long)a.score_stride, a.W);
+  if (a.rows > 1 && a.idx_stride < a.k)
+    return fail(QSA_ERR_INVALID_ARG, "idx_stride = %lld is below k = %d", (long long)a.idx_stride, a.k);
+  const Range ri = span(a.idx, 4, a.rows, a.idx_stride, 1, 0, 1, 0, a.k);
+  if (overlaps(ri, span(a.scores, 4, a.rows, a.score_stride, 1, 0, 1, 0, a.W)) ||
+      (a.lengths && overlaps(ri, span(a.lengths, 4, a.rows, 1, 1, 0, 1, 0, 1))))
+    return fail(QSA_ERR_INVALID_ARG, "idx overlaps an input");
+  return QSA_OK;
+}
+
+qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
+  int sms = 0;
+  qsa_status_t st = device_info(&sms);
+  if (st != QSA_OK) return st;
+  qsa::topk::Params p;
+  p.scores = a.scores;
+  p.stride = a.rows > 1 ? a.score_stride : a.W;
+  p.lengths = a.lengths;
+  p.W = a.W;
+  p.k = a.k;
+  p.idx = a.idx;
+  p.idx_stride = a.idx_stride;
+  p.vec4 = aligned(a.scores, 16) && (p.stride % 4 == 0);
+  if (a.W <= qsa::topk::MAX_CACHED_W) {
+    const size_t smem = sizeof(qsa::topk::Smem) + 4 * (size_t)a.W;
+    qsa::topk::topk_kernel<true><<<(unsigned)a.rows, qsa::topk::THREADS, smem, stream>>>(p);
+  } else {
+    qsa::topk::topk_kernel<false><<<(unsigned)a.rows, qsa::topk::THREADS, sizeof(qsa::topk::Smem), stream>>>(p);
+  }
+  return launch_status("top-k kernel");
+}
+
+}  // namespace
+
+// ================================================================ C ABI
+extern "C" {
+
+const char* qsa_status_string(qsa_status_t s) {
+  switch (s) {
+    case QSA_OK: return "QSA_OK";
+    case QSA_ERR_INVALID_ARG: return "QSA_ERR_INVALID_ARG: a size, count, pointer or value is out of range";
+    case QSA_ERR_ALIGNMENT: return "QSA_ERR_ALIGNMENT: a base address or stride breaks the layout rules";
+    case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED: configuration not implemented";
+    case QSA_ERR_WORKSPACE: return "QSA_ERR_WORKSPACE: workspace too small";
+    case QSA_ERR_CUDA: return "QSA_ERR_CUDA: CUDA call or launch failed";
+  }
+  return "unknown qsa_status_t";
+}
+
+const char* qsa_last_error_detail(void) { return g_detail; }
+
+qsa_status_t qsa_device_error(uint32_t* bits) {
+  if (!bits) return fail(QSA_ERR_INVALID_ARG, "bits must not be null");
+  unsigned int v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, qsa::g_device_error, sizeof v);
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(qsa::g_device_error, &zero, sizeof zero);
+  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+  *bits = v;
+  return ok();
+}
+
+qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
+                            const void* k_cache, int64_t num_pages, int32_t page_size, int64_t k_page_stride,
+                            int64_t k_row_stride, const int32_t* page_table, int64_t pt_stride, int32_t max_pages,
+                            const int32_t* seq_lens, int32_t B, int32_t Q, float scale, float* out,
+                            int64_t out_stride_b, int64_t out_stride_t, int32_t W, void* stream) {
+  if (B < 0 || W < 0) return fail(QSA_ERR_INVALID_ARG, "B and W must be non-negative");
+  if (Q < 1 || Q > 4) return fail(QSA_ERR_UNSUPPORTED, "Q = %d query tokens per request; 1..4 supported", Q);
+  if (page_size != 8 && page_size != 16 && page_size != 32 && page_size != 64)
+    return fail(QSA_ERR_UNSUPPORTED, "page_size = %d; supported page sizes are 8, 16, 32 and 64", page_size);
+  if (!std::isfinite(scale)) return fail(QSA_ERR_INVALID_ARG, "scale must be finite");
+  if (max_pages < 0) return fail(QSA_ERR_INVALID_ARG, "max_pages must be non-negative");
+  if (num_pages < 1 || num_pages > INT32_MAX)
+    return fail(QSA_ERR_INVALID_ARG, "num_pages = %lld must be in [1, 2^31 - 1]", (long long)num_pages);
+  if (B == 0 || W == 0) return ok();
+  if (!q || !k_cache || !seq_lens || !out || (max_pages > 0 && !page_table))
+    return fail(QSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(q, 16) || !aligned(k_cache, 16))
+    return fail(QSA_ERR_ALIGNMENT, "q and k_cache must be 16-byte aligned");
+  if (!aligned(out, 4) || !aligned(seq_lens, 4) || (page_table && !aligned(page_table, 4)))
+    return fail(QSA_ERR_ALIGNMENT, "out, seq_lens and page_table must be 4-byte aligned");
+  const int64_t qs[3] = {B > 1 ? q_stride_b : 0, Q > 1 ? q_stride_t : 0, q_stride_h};
+  for (int i = 0; i < 3; ++i)
+    if (qs[i] < 0 || qs[i] % 8 != 0)
+      return fail(QSA_ERR_ALIGNMENT, "q strides must be non-negative multiples of 8 (got %lld)", (long long)qs[i]);
+  if (k_row_stride < 128 || k_row_stride % 8 != 0)
+    return fail(QSA_ERR_ALIGNMENT, "k_row_stride = %lld must be a multiple of 8 and >= 128", (long long)k_row_stride);
+  if (num_pages > 1 && (k_page_stride <= 0 || k_page_stride % 8 != 0))
+    return fail(QSA_ERR_ALIGNMENT, "k_page_stride = %lld must be a positive multiple of 8", (long long)k_page_stride);
+  if (max_pages > 0 && B > 1 && pt_stride < max_pages)
+    return fail(QSA_ERR_INVALID_ARG, "pt_stride = %lld is below max_pages = %d", (long long)pt_stride, max_pages);
+  if (Q > 1 && out_stride_t < W) return fail(QSA_ERR_INVALID_ARG, "out_stride_t is below W");
+  if (B > 1 && out_stride_b < (int64_t)(Q - 1) * (Q > 1 ? out_stride_t : 0) + W)
+    return fail(QSA_ERR_INVALID_ARG, "out_stride_b is too small: rows of different requests overlap");
+  {
+    const Range ro = span(out, 4, B, B > 1 ? out_stride_b : 0, Q, Q > 1 ? out_stride_t : 0, 1, 0, W);
+    const Range rq = span(q, 2, B, qs[0], Q, qs[1], 4, qs[2], 128);
+    const Range rk = span(k_cache, 2, num_pages, num_pages > 1 ? k_page_stride : 0, page_size, k_row_stride, 1, 0, 128);
+    const Range rs = span(seq_lens, 4, B, 1, 1, 0, 1, 0, 1);
+    bool bad = overlaps(ro, rq) || overlaps(ro, rk) || overlaps(ro, rs);
+    if (max_pages > 0) bad = bad || overlaps(ro, span(page_table, 4, B, B > 1 ? pt_stride : 0, 1, 0, 1, 0, max_pages));
+    if (bad) return fail(QSA_ERR_INVALID_ARG, "out overlaps an input");
+  }
+
+  int sms = 0;
+  qsa_status_t st = device_info(&sms);
+  if (st != QSA_OK) return st;
+
+  CUtensorMap tm_k, tm_q;
+  {
+    cuuint64_t dims[3] = {128, (cuuint64_t)page_size, (cuuint64_t)num_pages};
+    const int64_t pstride = num_pages > 1 ? k_page_stride : (int64_t)page_size * k_row_stride;
+    cuuint64_t strides[2] = {(cuuint64_t)k_row_stride * 2, (cuuint64_t)pstride * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)page_size, 1};
+    st = encode_bf16_map(&tm_k, 3, const_cast<void*>(k_cache), dims, strides, box, "k_cache");
+    if (st != QSA_OK) return st;
+  }
+  qsa::decode::Params p;
+  p.q_bcast_h = q_stride_h == 0;
+  p.q_bcast_t = Q > 1 && q_stride_t == 0;
+  p.q_bcast_b = B > 1 && q_stride_b == 0;
+  p.q_mode = (p.q_bcast_h || p.q_bcast_t) ? 1 : 0;
+  {
+    const int64_t sh = p.q_bcast_h ? 128 : q_stride_h;
+    const int64_t dh = p.q_bcast_h ? 1 : 4;
+    const int64_t st_t = (Q > 1 && !p.q_bcast_t) ? q_stride_t : sh * dh;
+    const int64_t dt = (Q > 1 && !p.q_bcast_t) ? Q : 1;
+    const int64_t sb = (B > 1 && !p.q_bcast_b) ? q_stride_b : st_t * dt;
+    const int64_t db = (B > 1 && !p.q_bcast_b) ? B : 1;
+    cuuint64_t dims[4] = {128, (cuuint64_t)dh, (cuuint64_t)dt, (cuuint64_t)db};
+    cuuint64_t strides[3] = {(cuuint64_t)sh * 2, (cuuint64_t)st_t * 2, (cuuint64_t)sb * 2};
+    cuuint32_t box_full[4] = {64, 4, 4, 1}, box_row[4] = {64, 1, 1, 1};
+    st = encode_bf16_map(&tm_q, 4, const_cast<void*>(q), dims, strides, p.q_mode == 0 ? box_full : box_row, "q");
+    if (st != QSA_OK) return st;
+  }
+  p.page_table = page_table;
+  p.pt_stride = pt_stride;
+  p.max_pages = max_pages;
+  p.seq_lens = seq_lens;
+  p.B = B;
+  p.Q = Q;
+  p.log2_ps = page_size == 8 ? 3 : page_size == 16 ? 4 : page_size == 32 ? 5 : 6;
+  p.num_pages = num_pages;
+  p.scale = scale;
+  p.out = out;
+  p.out_sb = out_stride_b;
+  p.out_st = out_stride_t;
+  p.W = W;
+  qsa::decode::decode_kernel<<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES,
+                               static_cast<cudaStream_t>(stream)>>>(tm_k, tm_q, p);
+  return launch_status("decode kernel");
+}
+
+qsa_status_t qsa_mqa_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k, int64_t k_stride,
+                             int64_t Nk, const int32_t* ks, const int32_t* ke, int64_t T, float scale, float* out,
+                             int64_t out_stride, int32_t W, void* stream) {
+  PrefillArgs a{q, q_stride_t, q_stride_h, k, k_stride, Nk, ks, ke, T, scale, out, out_stride, W};
+  qsa_status_t st = validate_prefill(a);
+  if (st != QSA_OK) return st;
+  if (T == 0 || W == 0) return ok();
+  return launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+qsa_status_t qsa_prefill_intervals(const int32_t* cu_seqlens_q, const int32_t* seq_lens, const int32_t* key_offsets,
+                                   int32_t S, int64_t T, int32_t* ks, int32_t* ke, void* stream) {
+  if (S < 0 || T < 0) return fail(QSA_ERR_INVALID_ARG, "S and T must be non-negative");
+  if (T == 0) return ok();
+  if (S == 0) return fail(QSA_ERR_INVALID_ARG, "T > 0 rows need at least one sequence");
+  if (!cu_seqlens_q || !seq_lens || !key_offsets || !ks || !ke)
+    return fail(QSA_ERR_INVALID_ARG, "null pointer argument");
+  const int threads = 256;
+  const int64_t blocks = (T + threads - 1) / threads;
+  if (blocks > INT32_MAX) return fail(QSA_ERR_UNSUPPORTED, "T too large");
+  prefill_intervals_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      cu_seqlens_q, seq_lens, key_offsets, S, T, ks, ke);
+  return launch_status("prefill interval kernel");
+}
+
+qsa_status_t qsa_topk(const float* scores, int64_t score_stride, const int32_t* lengths, int64_t rows, int32_t W,
+                      int32_t k, int32_t* idx, int64_t idx_stride, void* stream) {
+  TopkArgs a{scores, score_stride, lengths, rows, W, k, idx, idx_stride};
+  qsa_status_t st = validate_topk(a);
+  if (st != QSA_OK) return st;
+  if (rows == 0) return ok();
+  return launch_topk(a, static_cast<cudaStream_t>(stream));
+}
+
+size_t qsa_prefill_topk_workspace_size(int64_t T, int32_t W) {
+  if (T <= 0 || W <= 0) return 0;
+  return (size_t)T * (size_t)W * sizeof(float);
+}
+
+qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
+                                  int64_t k_stride, int64_t Nk, const int32_t* ks, const int32_t* ke, int64_t T,
+                                  float scale, int32_t W, int32_t topk_k, int32_t* idx, int64_t idx_stride,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (W < 1) return fail(QSA_ERR_UNSUPPORTED, "W = %d must be in [1, 65536]", W);
+  float* ws = static_cast<float*>(workspace);
+  PrefillArgs pa{q, q_stride_t, q_stride_h, k, k_stride, Nk, ks, ke, T, scale, ws, (int64_t)W, W};
+  TopkArgs ta{ws, (int64_t)W, nullptr, T, W, topk_k, idx, idx_stride};
+  qsa_status_t st = validate_topk(ta);
+  if (st != QSA_OK) return st;
+  if (T < 0 || Nk < 0) return fail(QSA_ERR_INVALID_ARG, "T and Nk must be non-negative");
+  if (T == 0) return ok();
+  if (!workspace) return fail(QSA_ERR_WORKSPACE, "workspace is null");
+  if (!aligned(workspace, 16)) return fail(QSA_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  const int64_t row_bytes = (int64_t)W * 4;
+  int64_t chunk = (int64_t)(workspace_bytes / (size_t)row_bytes);
+  const int64_t min_rows = std::min<int64_t>(T, qsa::prefill::BT);
+  if (chunk < min_rows)
+    return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes holds %lld rows of W = %d floats; at least %lld needed",
+                workspace_bytes, (long long)chunk, W, (long long)min_rows);
+  if (chunk >= T) chunk = T;
+  else chunk = chunk / qsa::prefill::BT * qsa::prefill::BT;
+  {
+    // the workspace must not overlap anything the calls read or write
+    const Range rw = span(ws, 4, chunk, W, 1, 0, 1, 0, W);
+    const Range rq = span(q, 2, T, q_stride_t, 4, q_stride_h, 1, 0, 128);
+    const Range ri = span(idx, 4, T, idx_stride, 1, 0, 1, 0, topk_k);
+    bool bad = overlaps(rw, rq) || overlaps(rw, ri) || overlaps(rw, span(ks, 4, T, 1, 1, 0, 1, 0, 1)) ||
+               overlaps(rw, span(ke, 4, T, 1, 1, 0, 1, 0, 1));
+    if (Nk > 0) bad = bad || overlaps(rw, span(k, 2, Nk, k_stride, 1, 0, 1, 0, 128));
+    if (bad) return fail(QSA_ERR_INVALID_ARG, "workspace overlaps an input or idx");
+  }
+  for (int64_t r0 = 0; r0 < T; r0 += chunk) {
+    const int64_t n = std::min(chunk, T - r0);
+    PrefillArgs c = pa;
+    c.q = static_cast<const uint16_t*>(q) + r0 * q_stride_t;
+    c.ks = ks + r0;
+    c.ke = ke + r0;
+    c.T = n;
+    st = validate_prefill(c);
+    if (st != QSA_OK) return st;
+    st = launch_prefill(c, static_cast<cudaStream_t>(stream));
+    if (st != QSA_OK) return st;
+    TopkArgs t = ta;
+    t.rows = n;
+    t.idx = idx + r0 * idx_stride;
+    st = launch_topk(t, static_cast<cudaStream_t>(stream));
+    if (st != QSA_OK) return st;
+  }
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,136 @@
+"""The C-ABI library on a host without a GPU: it loads, exports every entry
+point include/qsa.h declares, and rejects bad arguments on the host before
+any CUDA call (no compute runs here)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import sparse_attention_block_qsa_b200 as qsa
+from sparse_attention_block_qsa_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qsa.h")
+
+OK, INVALID, ALIGN, UNSUP, WS = 0, 1, 2, 3, 4
+# fake device addresses: validation never dereferences them
+A = 0x7f0000000000
+S = 1 << 28        # distance between fake buffers
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qsa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 9
+    L = qsa.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (qsa_\w+)", out))
+    assert set(names) <= exported
+    assert set(names) == set(_abi.SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings():
+    L = qsa.lib()
+    for code in range(6):
+        assert L.qsa_status_string(code).decode().startswith(_abi.STATUS[code])
+
+
+def decode(**kw):
+    a = dict(q=A, sb=2048, st=512, sh=128, k=A + S, pages=100, ps=64, kps=64 * 128, krs=128, pt=A + 2 * S,
+             pts=10, maxp=10, sl=A + 3 * S, B=4, Q=4, scale=0.088, out=A + 4 * S, osb=4 * 1000, ost=1000, W=1000)
+    a.update(kw)
+    L = qsa.lib()
+    st = L.qsa_mqa_decode(a["q"], a["sb"], a["st"], a["sh"], a["k"], a["pages"], a["ps"], a["kps"], a["krs"],
+                          a["pt"], a["pts"], a["maxp"], a["sl"], a["B"], a["Q"], a["scale"], a["out"], a["osb"],
+                          a["ost"], a["W"], None)
+    return st, L.qsa_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Q=5), UNSUP), (dict(Q=0), UNSUP), (dict(ps=12), UNSUP), (dict(ps=128), UNSUP),
+    (dict(B=-1), INVALID), (dict(W=-1), INVALID), (dict(pages=0), INVALID), (dict(maxp=-1), INVALID),
+    (dict(scale=float("nan")), INVALID), (dict(q=0), INVALID), (dict(out=0), INVALID),
+    (dict(q=A + 2), ALIGN), (dict(k=A + S + 8), ALIGN), (dict(out=A + 4 * S + 2), ALIGN),
+    (dict(sh=100), ALIGN), (dict(st=-8), ALIGN), (dict(krs=120), ALIGN), (dict(kps=7), ALIGN),
+    (dict(pts=5), INVALID), (dict(ost=10), INVALID), (dict(osb=100), INVALID),
+    (dict(out=A + 100), INVALID),                      # out overlaps q
+])
+def test_decode_rejects(kw, code):
+    st, detail = decode(**kw)
+    assert st == code, detail
+    assert detail
+
+
+def test_decode_empty_batch_is_a_no_op():
+    assert decode(B=0)[0] == OK
+    assert decode(W=0)[0] == OK
+
+
+def prefill(**kw):
+    a = dict(q=A, st=512, sh=128, k=A + S, ks_=128, Nk=1000, ks=A + 2 * S, ke=A + 3 * S, T=100, scale=0.088,
+             out=A + 4 * S, os=2000, W=1000)
+    a.update(kw)
+    L = qsa.lib()
+    st = L.qsa_mqa_prefill(a["q"], a["st"], a["sh"], a["k"], a["ks_"], a["Nk"], a["ks"], a["ke"], a["T"],
+                           a["scale"], a["out"], a["os"], a["W"], None)
+    return st, L.qsa_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=-1), INVALID), (dict(Nk=-3), INVALID), (dict(W=-1), INVALID), (dict(T=1 << 31), UNSUP),
+    (dict(q=A + 8), ALIGN), (dict(k=A + S + 4), ALIGN), (dict(sh=0), ALIGN), (dict(st=0), ALIGN),
+    (dict(st=100), ALIGN), (dict(ks_=64), ALIGN), (dict(os=999), INVALID), (dict(ks=0), INVALID),
+    (dict(out=A + 2 * S), INVALID),                    # out overlaps ks
+    (dict(scale=float("inf")), INVALID),
+])
+def test_prefill_rejects(kw, code):
+    st, detail = prefill(**kw)
+    assert st == code, detail
+
+
+def test_prefill_empty_is_a_no_op():
+    assert prefill(T=0)[0] == OK
+    assert prefill(W=0)[0] == OK
+
+
+def topk(**kw):
+    a = dict(s=A, ss=5000, ln=0, rows=10, W=5000, k=512, idx=A + S, iss=512)
+    a.update(kw)
+    L = qsa.lib()
+    st = L.qsa_topk(a["s"], a["ss"], a["ln"] or None, a["rows"], a["W"], a["k"], a["idx"], a["iss"], None)
+    return st, L.qsa_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=0), UNSUP), (dict(k=2049), UNSUP), (dict(W=0), UNSUP), (dict(W=70000), UNSUP),
+    (dict(rows=-1), INVALID), (dict(ss=10), INVALID), (dict(iss=100), INVALID), (dict(s=A + 2), ALIGN),
+    (dict(idx=A + 4), INVALID),                         # idx overlaps scores
+])
+def test_topk_rejects(kw, code):
+    st, detail = topk(**kw)
+    assert st == code, detail
+
+
+def test_fused_rejects_small_workspace():
+    L = qsa.lib()
+    st = L.qsa_mqa_prefill_topk(A, 512, 128, A + S, 128, 1000, A + 2 * S, A + 3 * S, 1000, 0.088, 1000, 512,
+                                A + 4 * S, 512, A + 5 * S, 63 * 1000 * 4, None)
+    assert st == WS, L.qsa_last_error_detail().decode()
+    assert L.qsa_prefill_topk_workspace_size(16384, 26624) == 16384 * 26624 * 4
+
+
+def test_binding_refuses_cpu_tensors():
+    q = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        qsa.mqa_decode(q, torch.zeros(1, 16, 1, 128, dtype=torch.bfloat16), torch.zeros(1, 1, dtype=torch.int32),
+                       torch.zeros(1, dtype=torch.int32), 4)

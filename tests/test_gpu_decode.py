@@ -1,0 +1,114 @@
+"""Decode / spec-decode parity: the CUDA path through the C ABI against the
+fp64 oracle, element by element (B200 only)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from parity import compare_scores, decode_bounds
+
+pytestmark = pytest.mark.gpu
+
+qsa = pytest.importorskip("sparse_attention_block_qsa_b200")
+SCALE = 1.0 / np.sqrt(128.0)
+
+
+def run_case(d: wl.DecodeInputs, q=None, k_cache=None, out=None, W=None):
+    W = d.W if W is None else W
+    q = d.q if q is None else q
+    k_cache = d.k_cache if k_cache is None else k_cache
+    dev = torch.device("cuda")
+    res = qsa.mqa_decode(q.to(dev) if q.device.type == "cpu" else q, k_cache.to(dev) if k_cache.device.type == "cpu" else k_cache,
+                         d.page_table.to(dev), d.seq_lens.to(dev), W, scale=SCALE, out=out)
+    torch.cuda.synchronize()
+    assert qsa.device_error() == 0
+    gpu = res.cpu().numpy()
+    ref = oracle.decode(q.cpu(), k_cache.cpu(), d.page_table, d.seq_lens, W, scale=SCALE)
+    loose, tight = decode_bounds(q.cpu(), k_cache.cpu(), d.page_table, W, SCALE)
+    return compare_scores(gpu, ref, loose, tight)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_decode_full_config(cfg):
+    """The three decode workloads at full size, every output element."""
+    st = run_case(wl.make_config(cfg))
+    assert st["entries"] > 0
+
+
+@pytest.mark.parametrize("ps", [8, 16, 32, 64])
+@pytest.mark.parametrize("Q", [1, 2, 3, 4])
+def test_decode_ragged(ps, Q):
+    """Ragged lengths: empty, shorter than Q, not multiples of 4, spanning
+    several units and a partial last unit; W larger than every row needs."""
+    lens = [0, 1, 3, 4, 5, 7, 130, 511, 512, 513, 2049, 4 * 128 * 3 + 6]
+    d = wl.make_decode("ragged", lens, Q=Q, page_size=ps, seed=ps * 10 + Q, W=max(lens) // 4 + 37)
+    run_case(d)
+
+
+def test_decode_invalid_pages_and_short_table():
+    lens = [900, 1400, 333, 2000]
+    d = wl.make_decode("bad_pages", lens, Q=4, page_size=16, seed=7, table_pad=2)
+    t = d.page_table.clone()
+    P = d.k_cache.shape[0]
+    t[0, 1] = -1
+    t[1, 3] = P + 4            # past the pool
+    t[2, 0] = -7
+    t[3, 5:] = -1              # table ends early
+    d.page_table = t
+    run_case(d)
+    # a table with fewer columns than the visible keys need
+    d2 = wl.make_decode("short_table", [3000], Q=1, page_size=64, seed=8)
+    d2.page_table = d2.page_table[:, :5].contiguous()
+    run_case(d2)
+
+
+def test_decode_w_smaller_than_visible():
+    d = wl.make_decode("narrow", [5000, 60, 1200], Q=2, page_size=32, seed=9)
+    run_case(d, W=300)
+
+
+def test_decode_strided_views():
+    """Non-contiguous q / k_cache / out views that still meet the layout rules."""
+    d = wl.make_decode("strided", [777, 1500, 64], Q=3, page_size=32, seed=11)
+    dev = torch.device("cuda")
+    B, Q = d.B, d.Q
+    qbig = torch.zeros(B, Q + 1, 5, 136, dtype=torch.bfloat16)
+    qbig[:, :Q, :4, :128] = d.q
+    q = qbig.to(dev)[:, :Q, :4, :128]
+    P, ps = d.k_cache.shape[:2]
+    kbig = torch.zeros(P, ps + 3, 1, 144, dtype=torch.bfloat16)
+    kbig[:, :ps, :, :128] = d.k_cache
+    kc = kbig.to(dev)[:, :ps, :, :128]
+    out = torch.full((B, Q, d.W + 9), 7.0, device=dev)[:, :, :d.W]
+    run_case(d, q=q, k_cache=kc, out=out)
+
+
+@pytest.mark.parametrize("axis", ["b", "t", "h"])
+def test_decode_broadcast_query(axis):
+    """Stride-0 query axes (decode accepts broadcast queries)."""
+    d = wl.make_decode("bcast", [600, 1234, 99], Q=3, page_size=16, seed=12)
+    dev = torch.device("cuda")
+    base = d.q.to(dev)
+    if axis == "b":
+        q = base[:1].expand(d.B, -1, -1, -1)
+    elif axis == "t":
+        q = base[:, :1].expand(-1, d.Q, -1, -1)
+    else:
+        q = base[:, :, :1].expand(-1, -1, 4, -1)
+    run_case(d, q=q)
+
+
+def test_decode_repeat_is_bitwise_stable():
+    d = wl.make_config(2)
+    dev = torch.device("cuda")
+    args = (d.q.to(dev), d.k_cache.to(dev), d.page_table.to(dev), d.seq_lens.to(dev), d.W)
+    a = qsa.mqa_decode(*args).cpu()
+    b = qsa.mqa_decode(*args).cpu()
+    assert torch.equal(a, b)
+
+
+def test_decode_zero_queries_give_zero():
+    d = wl.make_decode("zero", [800, 333], Q=4, page_size=64, seed=13)
+    d.q = torch.zeros_like(d.q)
+    run_case(d)

@@ -110,9 +110,7 @@ qsa_status_t device_info(int* sms) {
     } kernels[] = {
         {reinterpret_cast<const void*>(qsa::decode::decode_kernel), qsa::decode::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel), qsa::prefill::SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::topk::topk_kernel<true>),
-         sizeof(qsa::topk::Smem) + 4 * (size_t)qsa::topk::MAX_CACHED_W},
-        {reinterpret_cast<const void*>(qsa::topk::topk_kernel<false>), sizeof(qsa::topk::Smem)},
+        {reinterpret_cast<const void*>(qsa::topk::topk_kernel), qsa::topk::SMEM_BYTES},
     };
     for (auto& k : kernels) {
       e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k.bytes);
@@ -280,12 +278,9 @@ qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   p.idx = a.idx;
   p.idx_stride = a.idx_stride;
   p.vec4 = aligned(a.scores, 16) && (p.stride % 4 == 0);
-  if (a.W <= qsa::topk::MAX_CACHED_W) {
-    const size_t smem = sizeof(qsa::topk::Smem) + 4 * (size_t)a.W;
-    qsa::topk::topk_kernel<true><<<(unsigned)a.rows, qsa::topk::THREADS, smem, stream>>>(p);
-  } else {
-    qsa::topk::topk_kernel<false><<<(unsigned)a.rows, qsa::topk::THREADS, sizeof(qsa::topk::Smem), stream>>>(p);
-  }
+  p.rows = a.rows;
+  const int64_t grid = std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::CTAS_PER_SM);
+  qsa::topk::topk_kernel<<<(unsigned)grid, qsa::topk::THREADS, qsa::topk::SMEM_BYTES, stream>>>(p);
   return launch_status("top-k kernel");
 }
 
@@ -365,49 +360,35 @@ qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_
   qsa_status_t st = device_info(&sms);
   if (st != QSA_OK) return st;
 
-  CUtensorMap tm_k, tm_q;
-  {
-    cuuint64_t dims[3] = {128, (cuuint64_t)page_size, (cuuint64_t)num_pages};
-    const int64_t pstride = num_pages > 1 ? k_page_stride : (int64_t)page_size * k_row_stride;
-    cuuint64_t strides[2] = {(cuuint64_t)k_row_stride * 2, (cuuint64_t)pstride * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)page_size, 1};
-    st = encode_bf16_map(&tm_k, 3, const_cast<void*>(k_cache), dims, strides, box, "k_cache");
-    if (st != QSA_OK) return st;
-  }
   qsa::decode::Params p;
-  p.q_bcast_h = q_stride_h == 0;
-  p.q_bcast_t = Q > 1 && q_stride_t == 0;
-  p.q_bcast_b = B > 1 && q_stride_b == 0;
-  p.q_mode = (p.q_bcast_h || p.q_bcast_t) ? 1 : 0;
-  {
-    const int64_t sh = p.q_bcast_h ? 128 : q_stride_h;
-    const int64_t dh = p.q_bcast_h ? 1 : 4;
-    const int64_t st_t = (Q > 1 && !p.q_bcast_t) ? q_stride_t : sh * dh;
-    const int64_t dt = (Q > 1 && !p.q_bcast_t) ? Q : 1;
-    const int64_t sb = (B > 1 && !p.q_bcast_b) ? q_stride_b : st_t * dt;
-    const int64_t db = (B > 1 && !p.q_bcast_b) ? B : 1;
-    cuuint64_t dims[4] = {128, (cuuint64_t)dh, (cuuint64_t)dt, (cuuint64_t)db};
-    cuuint64_t strides[3] = {(cuuint64_t)sh * 2, (cuuint64_t)st_t * 2, (cuuint64_t)sb * 2};
-    cuuint32_t box_full[4] = {64, 4, 4, 1}, box_row[4] = {64, 1, 1, 1};
-    st = encode_bf16_map(&tm_q, 4, const_cast<void*>(q), dims, strides, p.q_mode == 0 ? box_full : box_row, "q");
-    if (st != QSA_OK) return st;
-  }
-  p.page_table = page_table;
+  p.q_sb = B > 1 ? q_stride_b : 0;
+  p.q_st = Q > 1 ? q_stride_t : 0;
+  p.q_sh = q_stride_h;
+  p.k_cache = static_cast<const uint16_t*>(k_cache);
+  p.k_page_stride = num_pages > 1 ? k_page_stride : 0;
+  p.k_row_stride = k_row_stride;
+  p.num_pages = num_pages;
   p.pt_stride = pt_stride;
   p.max_pages = max_pages;
-  p.seq_lens = seq_lens;
-  p.B = B;
   p.Q = Q;
   p.log2_ps = page_size == 8 ? 3 : page_size == 16 ? 4 : page_size == 32 ? 5 : 6;
-  p.num_pages = num_pages;
   p.scale = scale;
-  p.out = out;
   p.out_sb = out_stride_b;
   p.out_st = out_stride_t;
   p.W = W;
-  qsa::decode::decode_kernel<<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES,
-                               static_cast<cudaStream_t>(stream)>>>(tm_k, tm_q, p);
-  return launch_status("decode kernel");
+  // requests are independent: launch them in groups that fit the kernel's prefix table
+  for (int32_t b0 = 0; b0 < B; b0 += qsa::decode::MAX_B) {
+    p.B = std::min(B - b0, qsa::decode::MAX_B);
+    p.q = static_cast<const uint16_t*>(q) + (int64_t)b0 * p.q_sb;
+    p.page_table = max_pages > 0 ? page_table + (int64_t)b0 * pt_stride : page_table;
+    p.seq_lens = seq_lens + b0;
+    p.out = out + (int64_t)b0 * out_stride_b;
+    qsa::decode::decode_kernel<<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES,
+                                 static_cast<cudaStream_t>(stream)>>>(p);
+    st = launch_status("decode kernel");
+    if (st != QSA_OK) return st;
+  }
+  return ok();
 }
 
 qsa_status_t qsa_mqa_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k, int64_t k_stride,

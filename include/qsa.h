@@ -184,9 +184,10 @@ qsa_status_t qsa_topk(const float* scores, int64_t score_stride, const int32_t* 
  * PR, "Main changes": prefill logits are bounded by a workspace limit and
  * processed chunk by chunk); each chunk runs qsa_mqa_prefill into the
  * workspace (row stride W) and then qsa_topk over it.  Arguments as for the
- * two calls; the result is idx only.  The workspace must hold at least
- * min(T, 128) rows of W floats and be 16-byte aligned;
- * qsa_prefill_topk_workspace_size gives the size that needs a single chunk.
+ * two calls; the result is idx only.  The workspace must be 16-byte aligned
+ * and hold 4096 bytes of selection state plus at least min(T, 64) rows of W
+ * floats; qsa_prefill_topk_workspace_size gives the size that needs a single
+ * chunk.
  * A workspace of a few tens of MB lets the chunk's scores stay in the
  * B200's 126 MB L2 between the two kernels.
  */

@@ -110,7 +110,8 @@ qsa_status_t device_info(int* sms) {
     } kernels[] = {
         {reinterpret_cast<const void*>(qsa::decode::decode_kernel), qsa::decode::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel), qsa::prefill::SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::topk::topk_kernel), qsa::topk::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::topk::topk_rows_kernel), qsa::topk::ROWS_SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::topk::topk_stream_kernel), qsa::topk::STREAM_SMEM_BYTES},
     };
     for (auto& k : kernels) {
       e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k.bytes);
@@ -265,7 +266,7 @@ qsa_status_t validate_topk(const TopkArgs& a) {
   return QSA_OK;
 }
 
-qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
+qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream, float* pred_state = nullptr) {
   int sms = 0;
   qsa_status_t st = device_info(&sms);
   if (st != QSA_OK) return st;
@@ -279,8 +280,16 @@ qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   p.idx_stride = a.idx_stride;
   p.vec4 = aligned(a.scores, 16) && (p.stride % 4 == 0);
   p.rows = a.rows;
-  const int64_t grid = std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::CTAS_PER_SM);
-  qsa::topk::topk_kernel<<<(unsigned)grid, qsa::topk::THREADS, qsa::topk::SMEM_BYTES, stream>>>(p);
+  p.pred_state = pred_state;
+  if (p.vec4 && a.W % 4 == 0) {
+    // rows start on 16-byte boundaries: stream them with bulk copies
+    const int64_t grid = std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::STREAM_CTAS_PER_SM);
+    qsa::topk::topk_stream_kernel<<<(unsigned)grid, qsa::topk::STREAM_THREADS, qsa::topk::STREAM_SMEM_BYTES,
+                                    stream>>>(p);
+  } else {
+    const int64_t grid = std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::ROWS_CTAS_PER_SM);
+    qsa::topk::topk_rows_kernel<<<(unsigned)grid, qsa::topk::THREADS, qsa::topk::ROWS_SMEM_BYTES, stream>>>(p);
+  }
   return launch_status("top-k kernel");
 }
 
@@ -427,7 +436,7 @@ qsa_status_t qsa_topk(const float* scores, int64_t score_stride, const int32_t* 
 
 size_t qsa_prefill_topk_workspace_size(int64_t T, int32_t W) {
   if (T <= 0 || W <= 0) return 0;
-  return (size_t)T * (size_t)W * sizeof(float);
+  return (size_t)T * (size_t)W * sizeof(float) + 4096;
 }
 
 qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
@@ -444,8 +453,15 @@ qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_s
   if (T == 0) return ok();
   if (!workspace) return fail(QSA_ERR_WORKSPACE, "workspace is null");
   if (!aligned(workspace, 16)) return fail(QSA_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  // the workspace ends with the top-k kernel's per-CTA predictions, carried
+  // from one chunk to the next
+  constexpr size_t kPredBytes = 4096;
+  if (workspace_bytes < kPredBytes)
+    return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes is too small", workspace_bytes);
+  const size_t score_bytes = (workspace_bytes - kPredBytes) & ~size_t(15);
+  float* pred_state = reinterpret_cast<float*>(static_cast<char*>(workspace) + score_bytes);
   const int64_t row_bytes = (int64_t)W * 4;
-  int64_t chunk = (int64_t)(workspace_bytes / (size_t)row_bytes);
+  int64_t chunk = (int64_t)(score_bytes / (size_t)row_bytes);
   const int64_t min_rows = std::min<int64_t>(T, qsa::prefill::BT);
   if (chunk < min_rows)
     return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes holds %lld rows of W = %d floats; at least %lld needed",
@@ -462,6 +478,10 @@ qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_s
     if (Nk > 0) bad = bad || overlaps(rw, span(k, 2, Nk, k_stride, 1, 0, 1, 0, 128));
     if (bad) return fail(QSA_ERR_INVALID_ARG, "workspace overlaps an input or idx");
   }
+  {
+    cudaError_t e = cudaMemsetAsync(pred_state, 0, kPredBytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+  }
   for (int64_t r0 = 0; r0 < T; r0 += chunk) {
     const int64_t n = std::min(chunk, T - r0);
     PrefillArgs c = pa;
@@ -476,7 +496,7 @@ qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_s
     TopkArgs t = ta;
     t.rows = n;
     t.idx = idx + r0 * idx_stride;
-    st = launch_topk(t, static_cast<cudaStream_t>(stream));
+    st = launch_topk(t, static_cast<cudaStream_t>(stream), pred_state);
     if (st != QSA_OK) return st;
   }
   return ok();

@@ -3,23 +3,32 @@
 // vLLM PR's review thread discusses).
 //
 // Persistent CTAs, each over a contiguous range of rows (neighbouring query
-// rows score alike).  Per row:
-//  * Fast path: one streaming read of the row (batched 16-byte loads); a
-//    float compare against a threshold predicted from the previous row's
-//    exact k-th value (x 0.9) and a warp ballot append the few scores above
-//    it to a shared-memory candidate list.  If that list holds at least k
-//    and at most CAP scores, it contains every selected column, and the
-//    exact selection runs on it alone.
-//  * Exact path (first row of a CTA, or a prediction that missed): a
-//    histogram of the top 13 bits of order-preserving keys over the row
-//    finds the bin holding the k-th key; a second read (from L2) marks every
-//    key of a higher bin and gathers the boundary bin into the list.  A
-//    pathological boundary bin (more than CAP keys) is narrowed with further
-//    passes over the row.
-//  * On the list, histogram levels over key bits (13, 10 and 9 bits) give
-//    the exact threshold key: keys above it are taken, keys equal to it are
-//    ties taken from the lowest column up.  A popcount scan over a column
-//    bitmap writes the selected columns in ascending order, then -1 padding.
+// rows score alike).  Two kernels share the selection logic:
+//  * topk_stream_kernel (rows 16-byte aligned, W a multiple of 4), two CTAs
+//    per SM: a producer warp streams every row of the CTA's range as 16 KB
+//    bulk copies into a 4-slot shared-memory ring without pausing between
+//    rows; 8 selecting warps read the ring.  While one CTA resolves a row,
+//    the other keeps streaming.
+//  * topk_rows_kernel (any alignment): 8 warps read each row with batched
+//    loads themselves.
+// Per row:
+//  * Fast path: every score is compared with a threshold predicted from an
+//    earlier row's exact k-th value (x 0.9); a lane holding a score at or
+//    above it appends it to its warp's segment of a candidate list (about 4%
+//    of the scores; the common case costs a compare per score).  If the list
+//    holds at least k scores and no segment overflowed, it holds every
+//    selected column and the selection runs on it alone: one histogram over
+//    [predicted key, largest key] finds the boundary bin; a warp ranks the
+//    boundary bin's keys (larger first, then lower column) when they are few,
+//    otherwise further histograms narrow the bin.
+//  * Exact path (no prediction yet, or one that missed): a histogram of the
+//    top 11 bits of order-preserving keys over the row finds the bin holding
+//    the k-th key; a second read of the row marks every key of a higher bin
+//    and gathers the boundary bin, resolved with 11- and 10-bit histograms; a
+//    pathological boundary bin is narrowed with further passes over the row.
+//    Its exact k-th value becomes the next prediction.
+//  * A popcount scan over a column bitmap writes the selected columns in
+//    ascending order, then -1 padding.
 // -inf and NaN scores are never candidates; -0.0 counts as +0.0.  The result
 // does not depend on the prediction, only the speed does.
 #pragma once
@@ -29,19 +38,25 @@
 namespace qsa {
 namespace topk {
 
-constexpr int THREADS = 512;
+constexpr int THREADS = 256;          // selecting threads (both kernels)
 constexpr int NWARPS = THREADS / 32;
-constexpr int CTAS_PER_SM = 2;
-constexpr int HBITS = 13;
+constexpr int ROWS_CTAS_PER_SM = 4;
+constexpr int STREAM_CTAS_PER_SM = 2;
+constexpr int HBITS = 11;
 constexpr int HBINS = 1 << HBITS;
 constexpr int HSHIFT = 32 - HBITS;
-constexpr int CAP = 4096;             // candidate list capacity
+constexpr int CAP = 2048;             // candidate list capacity
 constexpr int SEG = CAP / NWARPS;     // list slots owned by each warp
 constexpr int MAX_W = 65536;
 constexpr int BM_WORDS = MAX_W / 32;
-constexpr int NBINS_FINE = 1024;      // fallback narrowing histogram
+constexpr int NBINS_FINE = 1024;      // narrowing histogram
+constexpr int FBINS = 2048;           // fast-path histogram
 constexpr uint32_t ZERO_KEY = 0x80000000u;
 constexpr float PREDICT_MARGIN = 0.9f;
+constexpr int CHUNK = 4096;           // floats per ring slot (16 KB)
+constexpr int NST = 4;                // ring slots
+constexpr int STREAM_THREADS = THREADS + 32;
+static_assert(FBINS == HBINS, "the fast path and the exact path share one histogram");
 
 struct Params {
   const float* scores;
@@ -53,6 +68,7 @@ struct Params {
   int32_t* idx;
   int64_t idx_stride;
   int32_t vec4;            // rows are 16-byte aligned: use float4 loads
+  float* pred_state;       // per-CTA predictions carried between launches (may be null)
 };
 
 // Order-preserving key of a score; 0 marks "not a candidate".
@@ -68,27 +84,38 @@ __device__ __forceinline__ float key_value(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
-struct Smem {
+// Shared state of the selection (both kernels).
+struct Sel {
   uint32_t hist[HBINS];
   uint32_t gt[BM_WORDS];    // columns taken
   uint32_t tie[BM_WORDS];   // columns whose key equals the threshold
   uint32_t cand_key[CAP];
   int32_t cand_idx[CAP];
   uint32_t red[2 * NWARPS];
-  uint32_t seg_cnt[NWARPS];  // filled slots of each warp's segment
-  uint32_t n_cand;
+  uint32_t seg_cnt[NWARPS];  // keys appended by each warp (may pass SEG: overflow)
+  uint32_t small_key[32];
+  int32_t small_idx[32];
+  uint32_t n_small;
+  uint32_t kmax;
   uint32_t zeros;
   uint32_t total;
   uint32_t sel_bin;
   uint32_t sel_above;
   uint32_t lo, hi, need;
+  int abort;
+  int stop;  // abort as seen by the selecting warps at a row boundary
 };
 
-constexpr size_t SMEM_BYTES = sizeof(Smem);
+struct BlockSync {
+  __device__ static void sync() { __syncthreads(); }
+};
+struct ConsumerSync {  // the selecting threads only (the producer warp keeps streaming)
+  __device__ static void sync() { named_barrier_sync(1, THREADS); }
+};
 
-// Inclusive block scan of two counters; totals returned.
-__device__ __forceinline__ void block_scan2(uint32_t& a, uint32_t& b, uint32_t* red, uint32_t& ta,
-                                            uint32_t& tb) {
+// Inclusive scan of two counters over the selecting threads; totals returned.
+template <class Sync>
+__device__ __forceinline__ void block_scan2(uint32_t& a, uint32_t& b, uint32_t* red, uint32_t& ta, uint32_t& tb) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -103,7 +130,7 @@ __device__ __forceinline__ void block_scan2(uint32_t& a, uint32_t& b, uint32_t* 
     red[warp] = a;
     red[NWARPS + warp] = b;
   }
-  __syncthreads();
+  Sync::sync();
   uint32_t ba = 0, bb = 0;
   ta = 0;
   tb = 0;
@@ -117,14 +144,15 @@ __device__ __forceinline__ void block_scan2(uint32_t& a, uint32_t& b, uint32_t* 
     ta += ra;
     tb += rb;
   }
-  __syncthreads();
+  Sync::sync();
   a += ba;
   b += bb;
 }
 
-// Visit every column j < len with its score; all threads of the block take
-// every step together (columns past len arrive as -inf), so f may use
-// warp-collective operations.  Loads are issued in batches of 8 x 16 bytes.
+// Visit every column j < len of a row in global memory with its score; all
+// selecting threads take every step together (columns past len arrive as
+// -inf), so f may use warp-collective operations.  Loads are issued in
+// batches of 8 x 16 bytes.
 template <typename F>
 __device__ __forceinline__ void for_each_score(const Params& p, const float* row, int len, F&& f) {
   const int tid = threadIdx.x;
@@ -163,188 +191,81 @@ __device__ __forceinline__ void for_each_score(const Params& p, const float* row
   }
 }
 
-// Exact threshold among the candidate list (warp w's keys fill slots
-// [w * SEG, w * SEG + seg_cnt[w])): histogram levels over key bits [31:19],
-// [18:9] and [8:0], starting at `level` with the bits above it equal to
-// those of `lo`.  On return lo is the threshold key and nd the number of its
-// copies to take.
-__device__ __forceinline__ void resolve_list(Smem& S, int level, uint32_t& lo, uint32_t& nd) {
-  const int tid = threadIdx.x;
-#pragma unroll 1
-  for (; level < 3; ++level) {
-    const int shift = level == 0 ? 19 : level == 1 ? 9 : 0;
-    const int nbits = level == 0 ? 13 : level == 1 ? 10 : 9;
-    const uint32_t nb = 1u << nbits;
-    const uint32_t keep = level == 0 ? 0u : ~((1u << (shift + nbits)) - 1u);  // bits fixed so far
-    for (uint32_t i = tid; i < nb; i += THREADS) S.hist[i] = 0;
-    if (tid == 0) {
-      S.lo = lo;
-      S.need = nd;
-    }
-    __syncthreads();
-    for (uint32_t i = tid; i < CAP; i += THREADS) {
-      if ((i % SEG) >= S.seg_cnt[i / SEG]) continue;
-      const uint32_t key = S.cand_key[i];
-      if ((key & keep) == (lo & keep)) atomicAdd(&S.hist[(key >> shift) & (nb - 1u)], 1u);
-    }
-    __syncthreads();
-    const uint32_t per = nb / THREADS > 0 ? nb / THREADS : 1u;
-    uint32_t mine = 0;
-    if (tid * per < nb)
-      for (uint32_t i = 0; i < per; ++i) mine += S.hist[tid * per + i];
-    uint32_t incl = mine, dummy = 0, tot, td;
-    block_scan2(incl, dummy, S.red, tot, td);
-    const uint32_t above = tot - incl;  // keys in higher bins
-    if (above < nd && nd <= above + mine) {
-      uint32_t acc = above;
-      uint32_t bin = tid * per + per - 1;
-      while (acc + S.hist[bin] < nd) {
-        acc += S.hist[bin];
-        --bin;
-      }
-      S.lo = (lo & keep) | (bin << shift);
-      S.need = nd - acc;
-    }
-    __syncthreads();
-    lo = S.lo;
-    nd = S.need;
-    __syncthreads();
+// Fast path for one score: at or above the predicted (positive) threshold it
+// goes to this warp's list segment; its key is then simply the float bits
+// with the top bit set.
+__device__ __forceinline__ void fast_put(Sel& S, float x, int j, uint32_t& pos, uint32_t& kmax) {
+  const uint32_t key = __float_as_uint(x) | 0x80000000u;
+  const int warp = threadIdx.x >> 5;
+  if (pos < SEG) {
+    S.cand_key[warp * SEG + pos] = key;
+    S.cand_idx[warp * SEG + pos] = j;
+  }
+  kmax = max(kmax, key);
+  ++pos;
+}
+
+__device__ __forceinline__ void fast_visit4(Sel& S, float4 x, int j0, float pred, uint32_t& kmax) {
+  const bool h0 = x.x >= pred, h1 = x.y >= pred, h2 = x.z >= pred, h3 = x.w >= pred;
+  if (h0 | h1 | h2 | h3) {
+    uint32_t pos = atomicAdd(&S.seg_cnt[threadIdx.x >> 5], (uint32_t)h0 + h1 + h2 + h3);
+    if (h0) fast_put(S, x.x, j0, pos, kmax);
+    if (h1) fast_put(S, x.y, j0 + 1, pos, kmax);
+    if (h2) fast_put(S, x.z, j0 + 2, pos, kmax);
+    if (h3) fast_put(S, x.w, j0 + 3, pos, kmax);
   }
 }
 
-// Mark the list's keys above the threshold as taken and its threshold
-// copies as ties.
-__device__ __forceinline__ void mark_list(Smem& S, uint32_t thr) {
-  for (uint32_t i = threadIdx.x; i < CAP; i += THREADS) {
-    if ((i % SEG) >= S.seg_cnt[i / SEG]) continue;
-    const uint32_t key = S.cand_key[i];
-    const int32_t j = S.cand_idx[i];
-    if (key > thr) atomicOr(&S.gt[j >> 5], 1u << (j & 31));
-    else if (key == thr) atomicOr(&S.tie[j >> 5], 1u << (j & 31));
+__device__ __forceinline__ void fast_visit1(Sel& S, float x, int j, float pred, uint32_t& kmax) {
+  if (x >= pred) {
+    uint32_t pos = atomicAdd(&S.seg_cnt[threadIdx.x >> 5], 1u);
+    fast_put(S, x, j, pos, kmax);
   }
 }
 
-// Append (key, column) to this warp's list segment when `hit`; the count
-// lives in a register of every lane.  Returns false once the segment is
-// full (further keys are dropped and counted).
-__device__ __forceinline__ void warp_append(Smem& S, bool hit, uint32_t key, int j, uint32_t& count) {
+// Append (key, column) to this warp's list segment when `hit` (all lanes
+// call it together).
+__device__ __forceinline__ void warp_append(Sel& S, bool hit, uint32_t key, int j) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t m = __ballot_sync(0xffffffffu, hit);
   if (m) {
-    const uint32_t pos = count + __popc(m & ((1u << lane) - 1u));
+    uint32_t base = 0;
+    if (lane == 0) base = atomicAdd(&S.seg_cnt[warp], (uint32_t)__popc(m));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const uint32_t pos = base + __popc(m & ((1u << lane) - 1u));
     if (hit && pos < SEG) {
       S.cand_key[warp * SEG + pos] = key;
       S.cand_idx[warp * SEG + pos] = j;
     }
-    count += __popc(m);
   }
 }
 
-// Selection of one row into the bitmaps; returns the threshold key (0 when
-// every candidate is taken) and, in need_tie, how many of its copies count.
-__device__ __forceinline__ uint32_t select_row(const Params& p, Smem& S, const float* row, int len, float pred,
-                                               uint32_t& need_tie) {
-  const int tid = threadIdx.x, lane = tid & 31;
-  const uint32_t k = (uint32_t)p.k;
-  need_tie = 0;
-
-  // ---- fast path: gather the scores at or above the predicted threshold
-  if (pred > 0.f) {
-    uint32_t count = 0;
-    for_each_score(p, row, len, [&](int j, float x) {
-      const bool hit = x >= pred;
-      warp_append(S, hit, hit ? score_key(x) : 0u, j, count);
-    });
-    if (lane == 0) S.seg_cnt[threadIdx.x >> 5] = min(count, (uint32_t)SEG);
-    const uint32_t full = __reduce_or_sync(0xffffffffu, count > SEG ? 1u : 0u);
-    const uint32_t cnt = __reduce_add_sync(0xffffffffu, lane == 0 ? count : 0u);
-    if (lane == 0) {
-      atomicAdd(&S.n_cand, cnt);
-      if (full) atomicOr(&S.total, 0x80000000u);  // a segment overflowed
-    }
-    __syncthreads();
-    const uint32_t n = S.n_cand;
-    const bool overflow = S.total & 0x80000000u;
-    if (!overflow && n >= k) {
-      uint32_t lo = 0, nd = k;
-      resolve_list(S, 0, lo, nd);
-      mark_list(S, lo);
-      need_tie = nd;
-      return lo;
-    }
-    __syncthreads();  // everyone has read the counters before they are reset
-    if (tid == 0) {
-      S.n_cand = 0;
-      S.total = 0;
-    }
-    __syncthreads();
-  }
-
-  // ---- exact path, pass A: histogram of the top 13 key bits
-  uint32_t cnt = 0, zc = 0;
-  for_each_score(p, row, len, [&](int j, float x) {
-    const uint32_t key = score_key(x);
-    if (key) {
-      ++cnt;
-      if (key == ZERO_KEY) ++zc;
-      else atomicAdd(&S.hist[key >> HSHIFT], 1u);
-    }
-  });
-  cnt = __reduce_add_sync(0xffffffffu, cnt);
-  zc = __reduce_add_sync(0xffffffffu, zc);
-  if (lane == 0) {
-    atomicAdd(&S.total, cnt);
-    if (zc) atomicAdd(&S.zeros, zc);
-  }
-  __syncthreads();
-  if (tid == 0) S.hist[ZERO_KEY >> HSHIFT] += S.zeros;
-  __syncthreads();
-  const uint32_t total = S.total;
-  const bool take_all = total <= k;
-  if (!take_all) {
-    uint32_t mine = 0;  // thread t owns bins [16t, 16t + 16)
+// Keys in the list and whether a segment overflowed (read after a barrier).
+__device__ __forceinline__ uint32_t list_size(const Sel& S, bool& overflow) {
+  uint32_t n = 0;
+  overflow = false;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) mine += S.hist[16 * tid + i];
-    uint32_t incl = mine, dummy = 0, tot, td;
-    block_scan2(incl, dummy, S.red, tot, td);
-    const uint32_t above = tot - incl;
-    if (above < k && k <= above + mine) {
-      uint32_t acc = above;
-      int bin = 16 * tid + 15;
-      while (acc + S.hist[bin] < k) {
-        acc += S.hist[bin];
-        --bin;
-      }
-      S.sel_bin = (uint32_t)bin;
-      S.sel_above = acc;
-    }
-    __syncthreads();
+  for (int w = 0; w < NWARPS; ++w) {
+    n += S.seg_cnt[w];
+    overflow |= S.seg_cnt[w] > (uint32_t)SEG;
   }
-  const uint32_t sel_bin = take_all ? 0u : S.sel_bin;
-  const uint32_t need = take_all ? 0u : k - S.sel_above;  // keys to take from the boundary bin
+  return n;
+}
 
-  // ---- exact path, pass B: mark higher bins, gather the boundary bin
-  uint32_t count = 0;
-  for_each_score(p, row, len, [&](int j, float x) {
-    const uint32_t key = score_key(x);
-    const uint32_t bin = key >> HSHIFT;
-    if (key && (take_all || bin > sel_bin)) atomicOr(&S.gt[j >> 5], 1u << (j & 31));
-    warp_append(S, key && !take_all && bin == sel_bin, key, j, count);
-  });
-  if (lane == 0) S.seg_cnt[threadIdx.x >> 5] = min(count, (uint32_t)SEG);
-  const uint32_t full = __reduce_or_sync(0xffffffffu, count > SEG ? 1u : 0u);
-  if (lane == 0 && full) atomicOr(&S.n_cand, 1u);  // a segment overflowed
-  __syncthreads();
-  if (take_all) return 0u;
-  uint32_t lo = sel_bin << HSHIFT, nd = need;
-  if (S.n_cand == 0) {
-    resolve_list(S, 1, lo, nd);
-    mark_list(S, lo);
-    need_tie = nd;
-    return lo;
-  }
-  // narrow [lo, hi] inside the boundary bin until one key value is left
-  uint32_t hi = lo | ((1u << HSHIFT) - 1u);
+template <typename F>
+__device__ __forceinline__ void for_each_candidate(Sel& S, F&& f) {
+  for (uint32_t i = threadIdx.x; i < CAP; i += THREADS)
+    if ((i % SEG) < min(S.seg_cnt[i / SEG], (uint32_t)SEG)) f(S.cand_key[i], S.cand_idx[i]);
+}
+
+// Narrow [lo, hi] (keys of the candidate list, or of the row when row !=
+// nullptr) with 1024-bin histograms until one key value is left; nd is the
+// number of keys to take from the top of the range and on return the number
+// of threshold copies to take.
+template <class Sync>
+__device__ __forceinline__ void narrow(const Params& p, Sel& S, const float* row, int len, uint32_t& lo,
+                                       uint32_t& hi, uint32_t& nd) {
+  const int tid = threadIdx.x;
   for (int pass = 0; pass < 4 && lo < hi; ++pass) {
     const uint64_t span = (uint64_t)hi - lo + 1;
     int shift = 0;
@@ -355,108 +276,518 @@ __device__ __forceinline__ uint32_t select_row(const Params& p, Smem& S, const f
       S.hi = hi;
       S.need = nd;
     }
-    __syncthreads();
-    for_each_score(p, row, len, [&](int j, float x) {
-      const uint32_t key = score_key(x);
+    Sync::sync();
+    auto count = [&](uint32_t key) {
       if (key >= lo && key <= hi) atomicAdd(&S.hist[(key - lo) >> shift], 1u);
-    });
-    __syncthreads();
-    const uint32_t mine = S.hist[2 * tid] + S.hist[2 * tid + 1];
+    };
+    if (row) for_each_score(p, row, len, [&](int, float x) { count(score_key(x)); });
+    else for_each_candidate(S, [&](uint32_t key, int32_t) { count(key); });
+    Sync::sync();
+    constexpr int per = NBINS_FINE / THREADS;
+    uint32_t mine = 0;
+#pragma unroll
+    for (int i = 0; i < per; ++i) mine += S.hist[per * tid + i];
     uint32_t incl = mine, dummy = 0, tot, td;
-    block_scan2(incl, dummy, S.red, tot, td);
+    block_scan2<Sync>(incl, dummy, S.red, tot, td);
     const uint32_t above = tot - incl;
     if (above < nd && nd <= above + mine) {
       uint32_t acc = above;
-      int bin = 2 * tid + 1;
-      if (acc + S.hist[bin] < nd) {
+      int bin = per * tid + per - 1;
+      while (acc + S.hist[bin] < nd) {
         acc += S.hist[bin];
-        bin = 2 * tid;
+        --bin;
       }
       S.lo = lo + ((uint32_t)bin << shift);
       S.hi = (uint32_t)min((uint64_t)hi, (uint64_t)S.lo + ((uint64_t)1 << shift) - 1);
       S.need = nd - acc;
     }
-    __syncthreads();
+    Sync::sync();
     lo = S.lo;
     hi = S.hi;
     nd = S.need;
-    __syncthreads();
+    Sync::sync();
   }
   if (lo < hi && tid == 0) record_device_error(QSA_DEVERR_SELECT);
-  const uint32_t thr = lo, top = (sel_bin << HSHIFT) | ((1u << HSHIFT) - 1u);
-  for_each_score(p, row, len, [&](int j, float x) {
-    const uint32_t key = score_key(x);
-    if (key > thr && key <= top) atomicOr(&S.gt[j >> 5], 1u << (j & 31));
-    else if (key == thr && key) atomicOr(&S.tie[j >> 5], 1u << (j & 31));
-  });
-  need_tie = nd;
-  return thr;
 }
 
-__global__ void __launch_bounds__(THREADS, CTAS_PER_SM) topk_kernel(const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  Smem& S = *reinterpret_cast<Smem*>(smem_raw);
+// Bin of the k-th largest key of a 2048-bin histogram; thread t owns bins
+// [8t, 8t + 8).  Writes S.sel_bin and S.sel_above (keys in higher bins).
+template <class Sync>
+__device__ __forceinline__ void find_bin(Sel& S, uint32_t k) {
+  constexpr int per = HBINS / THREADS;
   const int tid = threadIdx.x;
+  uint32_t mine = 0;
+#pragma unroll
+  for (int i = 0; i < per; ++i) mine += S.hist[per * tid + i];
+  uint32_t incl = mine, dummy = 0, tot, td;
+  block_scan2<Sync>(incl, dummy, S.red, tot, td);
+  const uint32_t above = tot - incl;
+  if (above < k && k <= above + mine) {
+    uint32_t acc = above;
+    int bin = per * tid + per - 1;
+    while (acc + S.hist[bin] < k) {
+      acc += S.hist[bin];
+      --bin;
+    }
+    S.sel_bin = (uint32_t)bin;
+    S.sel_above = acc;
+  }
+  Sync::sync();
+}
+
+// Fast-path resolution on the candidate list (all keys >= key_lo, at least
+// k of them, S.hist zeroed): marks the selected columns.
+template <class Sync>
+__device__ __forceinline__ void resolve_candidates(const Params& p, Sel& S, uint32_t key_lo, uint32_t& thr,
+                                                   uint32_t& need_tie) {
+  const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t k = (uint32_t)p.k;
-  const int64_t r_begin = (int64_t)blockIdx.x * p.rows / gridDim.x;
-  const int64_t r_end = (int64_t)(blockIdx.x + 1) * p.rows / gridDim.x;
-  float pred = 0.f;  // predicted lower bound of the k-th score (0: none)
+  const uint32_t kmax = S.kmax;
+  const uint64_t span = (uint64_t)kmax - key_lo + 1;
+  int shift = 0;
+  while (((span - 1) >> shift) >= (uint64_t)FBINS) ++shift;
+  for_each_candidate(S, [&](uint32_t key, int32_t) { atomicAdd(&S.hist[(key - key_lo) >> shift], 1u); });
+  Sync::sync();
+  find_bin<Sync>(S, k);
+  const uint32_t B = S.sel_bin, nb = S.hist[B], needB = k - S.sel_above;
+  const uint32_t blo = key_lo + (B << shift);
+  const uint32_t bhi = (uint32_t)min((uint64_t)kmax, (uint64_t)blo + ((uint64_t)1 << shift) - 1);
+  // keys above the boundary bin are taken; its own keys are set aside
+  for_each_candidate(S, [&](uint32_t key, int32_t j) {
+    if (key > bhi) {
+      atomicOr(&S.gt[j >> 5], 1u << (j & 31));
+    } else if (key >= blo && nb <= 32) {
+      const uint32_t pos = atomicAdd(&S.n_small, 1u);
+      S.small_key[pos] = key;
+      S.small_idx[pos] = j;
+    }
+  });
+  Sync::sync();
+  if (nb <= 32) {
+    if (tid < 32) {  // one warp ranks the boundary keys: larger first, then lower column
+      const bool have = (uint32_t)lane < nb;
+      const uint32_t key = have ? S.small_key[lane] : 0u;
+      const int32_t j = have ? S.small_idx[lane] : INT32_MAX;
+      uint32_t rank = 0;
+      for (int o = 0; o < 32; ++o) {
+        const uint32_t ko = __shfl_sync(0xffffffffu, key, o);
+        const int32_t jo = __shfl_sync(0xffffffffu, j, o);
+        rank += (ko > key) || (ko == key && jo < j);
+      }
+      if (have && rank < needB) atomicOr(&S.gt[j >> 5], 1u << (j & 31));
+    }
+    thr = 0;
+    need_tie = 0;
+    return;
+  }
+  uint32_t lo = blo, hi = bhi, nd = needB;
+  narrow<Sync>(p, S, nullptr, 0, lo, hi, nd);
+  for_each_candidate(S, [&](uint32_t key, int32_t j) {
+    if (key > lo && key <= bhi) atomicOr(&S.gt[j >> 5], 1u << (j & 31));
+    else if (key == lo) atomicOr(&S.tie[j >> 5], 1u << (j & 31));
+  });
+  thr = lo;
+  need_tie = nd;
+}
 
-  for (int64_t r = r_begin; r < r_end; ++r) {
-    const float* row = p.scores + r * p.stride;
-    int32_t* out = p.idx + r * p.idx_stride;
-    int len = p.W;
-    if (p.lengths != nullptr) len = min(max(__ldg(p.lengths + r), 0), p.W);
-    const int nwords = (len + 31) >> 5;
-
-    for (int i = tid; i < HBINS; i += THREADS) S.hist[i] = 0;
-    for (int i = tid; i < nwords; i += THREADS) S.gt[i] = S.tie[i] = 0;
+// Exact threshold among the list keys of the boundary bin: histogram levels
+// over key bits [20:10] and [9:0] below the bin's 11 bits.
+template <class Sync>
+__device__ __forceinline__ void resolve_bin(Sel& S, uint32_t& lo, uint32_t& nd) {
+  const int tid = threadIdx.x;
+#pragma unroll 1
+  for (int level = 0; level < 2; ++level) {
+    const int shift = level == 0 ? 10 : 0;
+    const int nbits = level == 0 ? 11 : 10;
+    const uint32_t nb = 1u << nbits;
+    const uint32_t keep = ~((1u << (shift + nbits)) - 1u);  // bits fixed so far
+    for (uint32_t i = tid; i < nb; i += THREADS) S.hist[i] = 0;
     if (tid == 0) {
-      S.n_cand = 0;
+      S.lo = lo;
+      S.need = nd;
+    }
+    Sync::sync();
+    for_each_candidate(S, [&](uint32_t key, int32_t) {
+      if ((key & keep) == (lo & keep)) atomicAdd(&S.hist[(key >> shift) & (nb - 1u)], 1u);
+    });
+    Sync::sync();
+    const uint32_t per = nb / THREADS;
+    uint32_t mine = 0;
+    for (uint32_t i = 0; i < per; ++i) mine += S.hist[tid * per + i];
+    uint32_t incl = mine, dummy = 0, tot, td;
+    block_scan2<Sync>(incl, dummy, S.red, tot, td);
+    const uint32_t above = tot - incl;
+    if (above < nd && nd <= above + mine) {
+      uint32_t acc = above;
+      uint32_t bin = tid * per + per - 1;
+      while (acc + S.hist[bin] < nd) {
+        acc += S.hist[bin];
+        --bin;
+      }
+      S.lo = (lo & keep) | (bin << shift);
+      S.need = nd - acc;
+    }
+    Sync::sync();
+    lo = S.lo;
+    nd = S.need;
+    Sync::sync();
+  }
+}
+
+// Exact selection reading the row from global memory; when have_hist the
+// 11-bit histogram of the row (pass A) is already in S.hist / S.total.
+template <class Sync>
+__device__ __forceinline__ void exact_select(const Params& p, Sel& S, const float* row, int len, bool have_hist,
+                                             uint32_t& thr, uint32_t& need_tie) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t k = (uint32_t)p.k;
+  thr = 0;
+  need_tie = 0;
+  if (!have_hist) {
+    for (int i = tid; i < HBINS; i += THREADS) S.hist[i] = 0;
+    if (tid == 0) {
       S.zeros = 0;
       S.total = 0;
     }
-    __syncthreads();
+    Sync::sync();
+    uint32_t cnt = 0, zc = 0;
+    for_each_score(p, row, len, [&](int, float x) {
+      const uint32_t key = score_key(x);
+      if (key) {
+        ++cnt;
+        if (key == ZERO_KEY) ++zc;
+        else atomicAdd(&S.hist[key >> HSHIFT], 1u);
+      }
+    });
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    zc = __reduce_add_sync(0xffffffffu, zc);
+    if (lane == 0) {
+      atomicAdd(&S.total, cnt);
+      if (zc) atomicAdd(&S.zeros, zc);
+    }
+    Sync::sync();
+  }
+  if (tid == 0) S.hist[ZERO_KEY >> HSHIFT] += S.zeros;
+  if (tid < NWARPS) S.seg_cnt[tid] = 0;
+  Sync::sync();
+  const uint32_t total = S.total;
+  const bool take_all = total <= k;
+  if (!take_all) find_bin<Sync>(S, k);
+  const uint32_t sel_bin = take_all ? 0u : S.sel_bin;
+  const uint32_t need = take_all ? 0u : k - S.sel_above;  // keys to take from the boundary bin
+  // pass B: mark higher bins, gather the boundary bin
+  for_each_score(p, row, len, [&](int j, float x) {
+    const uint32_t key = score_key(x);
+    const uint32_t bin = key >> HSHIFT;
+    if (key && (take_all || bin > sel_bin)) atomicOr(&S.gt[j >> 5], 1u << (j & 31));
+    warp_append(S, key && !take_all && bin == sel_bin, key, j);
+  });
+  Sync::sync();
+  if (take_all) return;
+  bool overflow;
+  list_size(S, overflow);
+  uint32_t lo = sel_bin << HSHIFT, nd = need;
+  const uint32_t top = lo | ((1u << HSHIFT) - 1u);
+  if (!overflow) {
+    resolve_bin<Sync>(S, lo, nd);
+  } else {
+    uint32_t hi = top;
+    narrow<Sync>(p, S, row, len, lo, hi, nd);
+  }
+  auto mark = [&](uint32_t key, int32_t j) {
+    if (key > lo && key <= top) atomicOr(&S.gt[j >> 5], 1u << (j & 31));
+    else if (key == lo && key) atomicOr(&S.tie[j >> 5], 1u << (j & 31));
+  };
+  if (!overflow) for_each_candidate(S, mark);
+  else for_each_score(p, row, len, [&](int j, float x) { mark(score_key(x), j); });
+  thr = lo;
+  need_tie = nd;
+}
 
-    uint32_t need_tie;
-    const uint32_t thr = select_row(p, S, row, len, pred, need_tie);
-    __syncthreads();
-    // next row: a little below this row's k-th score (positive scores only)
-    const float tv = thr ? key_value(thr) : 0.f;
-    pred = (thr & 0x80000000u) && tv > 0.f ? tv * PREDICT_MARGIN : 0.f;
-
-    // ---- ordered output: contiguous bitmap words per thread
-    const int wpt = (nwords + THREADS - 1) / THREADS;
-    const int w0 = min(tid * wpt, nwords), w1 = min(w0 + wpt, nwords);
-    uint32_t ties = 0;
-    for (int w = w0; w < w1; ++w) ties += __popc(S.tie[w]);
-    uint32_t t_incl = ties, d0 = 0, t_tot, d_tot;
-    block_scan2(t_incl, d0, S.red, t_tot, d_tot);
+// Bitmap -> ascending column list (ties beyond need_tie dropped from the top),
+// -1 padding; the bitmap words are cleared for the next row on the way.
+template <class Sync>
+__device__ __forceinline__ void write_row(const Params& p, Sel& S, int32_t* out, int nwords, uint32_t need_tie) {
+  const int tid = threadIdx.x;
+  const uint32_t k = (uint32_t)p.k;
+  const int wpt = (nwords + THREADS - 1) / THREADS;
+  const int w0 = min(tid * wpt, nwords), w1 = min(w0 + wpt, nwords);
+  uint32_t ties = 0, sel = 0;
+  for (int w = w0; w < w1; ++w) {
+    ties += __popc(S.tie[w]);
+    sel += __popc(S.gt[w]);
+  }
+  uint32_t t_incl = ties, g_incl = sel, t_tot, g_tot;
+  block_scan2<Sync>(t_incl, g_incl, S.red, t_tot, g_tot);
+  uint32_t pos, s_tot = g_tot;
+  if (t_tot > 0) {  // keep the lowest need_tie ties
     const uint32_t ties_before = t_incl - ties;
-    uint32_t tie_left = need_tie > ties_before ? need_tie - ties_before : 0u;  // ties this thread may take
-    uint32_t sel = 0;
+    uint32_t tie_left = need_tie > ties_before ? need_tie - ties_before : 0u;
+    sel = 0;
     for (int w = w0; w < w1; ++w) {
       uint32_t tw = S.tie[w];
-      while (tw && (uint32_t)__popc(tw) > tie_left) tw &= ~(1u << (31 - __clz(tw)));  // keep the lowest
+      while (tw && (uint32_t)__popc(tw) > tie_left) tw &= ~(1u << (31 - __clz(tw)));
       tie_left -= (uint32_t)__popc(tw);
       S.tie[w] = tw;
       sel += (uint32_t)__popc(S.gt[w] | tw);
     }
-    uint32_t s_incl = sel, d1 = 0, s_tot, d1_tot;
-    block_scan2(s_incl, d1, S.red, s_tot, d1_tot);
-    uint32_t pos = s_incl - sel;
-    for (int w = w0; w < w1; ++w) {
-      uint32_t bits = S.gt[w] | S.tie[w];
-      while (bits) {
-        const int b = __ffs(bits) - 1;
-        bits &= bits - 1;
-        if (pos < k) out[pos] = w * 32 + b;
-        ++pos;
-      }
-    }
-    for (uint32_t s = min(s_tot, k) + tid; s < k; s += THREADS) out[s] = -1;
-    __syncthreads();  // bitmaps and histogram are reused by the next row
+    uint32_t s_incl = sel, d1 = 0, d1_tot;
+    block_scan2<Sync>(s_incl, d1, S.red, s_tot, d1_tot);
+    pos = s_incl - sel;
+  } else {
+    pos = g_incl - sel;
   }
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = S.gt[w] | S.tie[w];
+    S.gt[w] = 0;
+    S.tie[w] = 0;
+    while (bits) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (pos < k) out[pos] = w * 32 + b;
+      ++pos;
+    }
+  }
+  for (uint32_t s = min(s_tot, k) + tid; s < k; s += THREADS) out[s] = -1;
+}
+
+__device__ __forceinline__ float next_prediction(uint32_t thr) {
+  const float tv = thr ? key_value(thr) : 0.f;
+  return (thr & 0x80000000u) && tv > 0.f ? tv * PREDICT_MARGIN : 0.f;
+}
+
+__device__ __forceinline__ int row_len(const Params& p, int64_t r) {
+  return p.lengths != nullptr ? min(max(__ldg(p.lengths + r), 0), p.W) : p.W;
+}
+
+// Reset the per-row state that the fast path relies on (before a barrier).
+__device__ __forceinline__ void start_row(Sel& S) {
+  const int tid = threadIdx.x;
+  for (int i = tid; i < HBINS; i += THREADS) S.hist[i] = 0;
+  if (tid < NWARPS) S.seg_cnt[tid] = 0;
+  if (tid == 0) {
+    S.kmax = 0;
+    S.zeros = 0;
+    S.total = 0;
+    S.n_small = 0;
+  }
+}
+
+// -------------------------------------------------------------- general kernel
+
+__global__ void __launch_bounds__(THREADS, ROWS_CTAS_PER_SM) topk_rows_kernel(const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Sel& S = *reinterpret_cast<Sel*>(smem_raw);
+  const int tid = threadIdx.x;
+  const uint32_t k = (uint32_t)p.k;
+  const int64_t r_begin = (int64_t)blockIdx.x * p.rows / gridDim.x;
+  const int64_t r_end = (int64_t)(blockIdx.x + 1) * p.rows / gridDim.x;
+  float pred = p.pred_state ? p.pred_state[blockIdx.x] : 0.f;
+  for (int i = tid; i < BM_WORDS; i += THREADS) S.gt[i] = S.tie[i] = 0;
+
+  for (int64_t r = r_begin; r < r_end; ++r) {
+    const float* row = p.scores + r * p.stride;
+    const int len = row_len(p, r);
+    start_row(S);
+    __syncthreads();
+    uint32_t thr = 0, need_tie = 0;
+    bool done = false;
+    if (pred > 0.f) {
+      uint32_t kmax = 0;
+      for_each_score(p, row, len, [&](int j, float x) { fast_visit1(S, x, j, pred, kmax); });
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      if ((tid & 31) == 0) atomicMax(&S.kmax, kmax);
+      __syncthreads();
+      bool overflow;
+      if (list_size(S, overflow) >= k && !overflow) {
+        resolve_candidates<BlockSync>(p, S, __float_as_uint(pred) | 0x80000000u, thr, need_tie);
+        done = true;
+      }
+      __syncthreads();
+    }
+    if (!done) exact_select<BlockSync>(p, S, row, len, false, thr, need_tie);
+    __syncthreads();
+    if (!done) pred = next_prediction(thr);  // a miss refreshes the prediction
+    write_row<BlockSync>(p, S, p.idx + r * p.idx_stride, (len + 31) >> 5, need_tie);
+    __syncthreads();
+  }
+  if (p.pred_state && tid == 0) p.pred_state[blockIdx.x] = pred;
+}
+
+// -------------------------------------------------------------- streaming kernel
+
+struct StreamSmem {
+  float ring[NST * CHUNK];
+  uint64_t full[NST];
+  uint64_t empty[NST];
+  Sel sel;
+};
+
+constexpr size_t STREAM_SMEM_BYTES = sizeof(StreamSmem) + 128;
+constexpr size_t ROWS_SMEM_BYTES = sizeof(Sel);
+
+__global__ void __launch_bounds__(STREAM_THREADS, STREAM_CTAS_PER_SM) topk_stream_kernel(const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  StreamSmem& M = *reinterpret_cast<StreamSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  Sel& S = M.sel;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t k = (uint32_t)p.k;
+  const int64_t r_begin = (int64_t)blockIdx.x * p.rows / gridDim.x;
+  const int64_t r_end = (int64_t)(blockIdx.x + 1) * p.rows / gridDim.x;
+
+  if (tid == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&M.full[s], 1);
+      mbar_init(&M.empty[s], NWARPS);
+    }
+    S.abort = 0;
+    fence_mbar_init();
+  }
+  for (int i = tid; i < BM_WORDS; i += STREAM_THREADS) S.gt[i] = S.tie[i] = 0;
+  __syncthreads();
+
+  if (warp == NWARPS) {
+    // ================= producer: every chunk of every row, back to back
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int64_t r = r_begin; r < r_end && !*(volatile int*)&S.abort; ++r) {
+        const int len4 = (row_len(p, r) + 3) & ~3;  // within the row: W is a multiple of 4
+        const float* row = p.scores + r * p.stride;
+        for (int c0 = 0; c0 < len4; c0 += CHUNK, ++it) {
+          const int s = it % NST;
+          if (!mbar_wait(&M.empty[s], ((it / NST) & 1) ^ 1, &S.abort)) {
+            if (atomicExch(&S.abort, 1) == 0) record_device_error(QSA_DEVERR_WAIT_TIMEOUT);
+            break;
+          }
+          const uint32_t bytes = (uint32_t)min(CHUNK, len4 - c0) * 4u;
+          mbar_arrive_expect_tx(&M.full[s], bytes);
+          asm volatile(
+              "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                  smem_addr(M.ring + s * CHUNK)),
+              "l"(row + c0), "r"(bytes), "r"(smem_addr(&M.full[s]))
+              : "memory");
+        }
+      }
+      // the last copy into every slot must land before the block may retire
+      for (uint32_t i = it > (uint32_t)NST ? it - NST : 0u; i < it; ++i)
+        if (!mbar_wait(&M.full[i % NST], (i / NST) & 1, nullptr)) break;
+    }
+    __syncwarp();
+    return;  // the selecting threads never wait for this warp
+  }
+
+  // ================= 8 selecting warps
+  float pred = p.pred_state ? p.pred_state[blockIdx.x] : 0.f;
+  uint32_t it = 0;
+  for (int64_t r = r_begin; r < r_end; ++r) {
+    const float* row = p.scores + r * p.stride;
+    const int len = row_len(p, r);
+    const int len4 = (len + 3) & ~3;
+    const bool fast = pred > 0.f;
+    start_row(S);
+    ConsumerSync::sync();
+    uint32_t kmax = 0, cnt = 0, zc = 0;
+    uint32_t count = 0;  // this warp's list entries (warp-uniform)
+    for (int c0 = 0; c0 < len4; c0 += CHUNK, ++it) {
+      const int s = it % NST;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&M.full[s], (it / NST) & 1, &S.abort));
+      if (ok) {
+        const float4* ring4 = reinterpret_cast<const float4*>(M.ring + s * CHUNK);
+        const bool tail = c0 + CHUNK > len;
+        uint32_t mask = 0;  // fast path: bit 4u + e = score e of this lane's u-th float4 is a candidate
+#pragma unroll
+        for (int u = 0; u < CHUNK / 4 / THREADS; ++u) {
+          const int f = u * THREADS + tid;
+          float4 x = ring4[f];
+          const int j0 = c0 + 4 * f;
+          if (tail) {
+            if (j0 >= len) x.x = -INFINITY;
+            if (j0 + 1 >= len) x.y = -INFINITY;
+            if (j0 + 2 >= len) x.z = -INFINITY;
+            if (j0 + 3 >= len) x.w = -INFINITY;
+          }
+          if (fast) {
+            mask |= (uint32_t)(x.x >= pred) << (4 * u) | (uint32_t)(x.y >= pred) << (4 * u + 1) |
+                    (uint32_t)(x.z >= pred) << (4 * u + 2) | (uint32_t)(x.w >= pred) << (4 * u + 3);
+          } else {
+            const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t key = score_key(xs[e]);
+              if (key) {
+                ++cnt;
+                if (key == ZERO_KEY) ++zc;
+                else atomicAdd(&S.hist[key >> HSHIFT], 1u);
+              }
+            }
+          }
+        }
+        if (fast) {
+          // positions from a warp scan of the lanes' candidate counts; then
+          // each lane copies its few candidates from the ring into the list
+          const uint32_t nl = __popc(mask);
+          uint32_t incl = nl;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          uint32_t pos = count + incl - nl;
+          count += __shfl_sync(0xffffffffu, incl, 31);
+          while (mask) {
+            const int b = __ffs(mask) - 1;
+            mask &= mask - 1;
+            const int f = (b >> 2) * THREADS + tid;
+            const float x = M.ring[s * CHUNK + 4 * f + (b & 3)];
+            const uint32_t key = __float_as_uint(x) | 0x80000000u;  // x >= pred > 0
+            if (pos < SEG) {
+              S.cand_key[warp * SEG + pos] = key;
+              S.cand_idx[warp * SEG + pos] = c0 + 4 * f + (b & 3);
+            }
+            kmax = max(kmax, key);
+            ++pos;
+          }
+        }
+      } else if (lane == 0 && atomicExch(&S.abort, 1) == 0) {
+        record_device_error(QSA_DEVERR_WAIT_TIMEOUT);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&M.empty[s]);
+    }
+    uint32_t thr = 0, need_tie = 0;
+    bool done = false;
+    if (fast) {
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      if (lane == 0) {
+        atomicMax(&S.kmax, kmax);
+        S.seg_cnt[warp] = count;
+      }
+      ConsumerSync::sync();
+      bool overflow;
+      if (list_size(S, overflow) >= k && !overflow) {
+        resolve_candidates<ConsumerSync>(p, S, __float_as_uint(pred) | 0x80000000u, thr, need_tie);
+        done = true;
+      }
+      ConsumerSync::sync();
+      if (!done) exact_select<ConsumerSync>(p, S, row, len, false, thr, need_tie);
+    } else {
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      zc = __reduce_add_sync(0xffffffffu, zc);
+      if (lane == 0) {
+        atomicAdd(&S.total, cnt);
+        if (zc) atomicAdd(&S.zeros, zc);
+      }
+      ConsumerSync::sync();
+      exact_select<ConsumerSync>(p, S, row, len, true, thr, need_tie);
+    }
+    ConsumerSync::sync();
+    if (!done) pred = next_prediction(thr);  // a miss refreshes the prediction
+    write_row<ConsumerSync>(p, S, p.idx + r * p.idx_stride, (len + 31) >> 5, need_tie);
+    if (tid == 0) S.stop = *(volatile int*)&S.abort;  // one reading for every warp
+    ConsumerSync::sync();
+    if (S.stop) break;
+  }
+  if (p.pred_state && tid == 0) p.pred_state[blockIdx.x] = pred;
 }
 
 }  // namespace topk

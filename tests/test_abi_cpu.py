@@ -126,7 +126,7 @@ def test_fused_rejects_small_workspace():
     st = L.qsa_mqa_prefill_topk(A, 512, 128, A + S, 128, 1000, A + 2 * S, A + 3 * S, 1000, 0.088, 1000, 512,
                                 A + 4 * S, 512, A + 5 * S, 63 * 1000 * 4, None)
     assert st == WS, L.qsa_last_error_detail().decode()
-    assert L.qsa_prefill_topk_workspace_size(16384, 26624) == 16384 * 26624 * 4
+    assert L.qsa_prefill_topk_workspace_size(16384, 26624) == 16384 * 26624 * 4 + 4096
 
 
 def test_binding_refuses_cpu_tensors():

@@ -198,6 +198,35 @@ qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_s
 
 size_t qsa_prefill_topk_workspace_size(int64_t T, int32_t W);
 
+/*
+ * qsa_mqa_prefill_topk_noalloc - qsa_mqa_prefill_topk without a caller
+ * workspace.
+ *
+ * The pages have no counterpart to this call.  It is for callers that cannot
+ * allocate device memory at call time: a host program whose device memory is
+ * planned up front by a framework that hands out fixed pools, or code on a
+ * thread where cudaMalloc is not allowed because it may synchronise the
+ * device.  The scores pass through a 16 MiB static array compiled into this
+ * library (every GPU that loads the library keeps it until the process
+ * exits); no cudaMalloc, cudaFree or allocating library routine is called.
+ * Arguments and results as for qsa_mqa_prefill_topk.
+ *
+ *  - One chunk of min(T, 64) rows of W floats plus 4096 bytes of selection
+ *    state must fit in the 16 MiB: larger W returns QSA_ERR_WORKSPACE
+ *    (W <= 65520 always fits).  Longer batches are processed in more chunks.
+ *  - The first call on a device, with that device current, looks up the
+ *    array's device address (cudaGetSymbolAddress); make that first call
+ *    before any stream capture.
+ *  - All calls share the array, which keeps the last call's contents; the
+ *    call clears the part that must start at zero.  Calls that overlap on
+ *    the GPU (different streams, or different host threads on one device)
+ *    race on the array and must be serialised by the caller.
+ */
+qsa_status_t qsa_mqa_prefill_topk_noalloc(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
+                                          int64_t k_stride, int64_t Nk, const int32_t* ks, const int32_t* ke,
+                                          int64_t T, float scale, int32_t W, int32_t topk_k, int32_t* idx,
+                                          int64_t idx_stride, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

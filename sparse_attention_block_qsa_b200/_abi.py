@@ -32,6 +32,8 @@ SIGNATURES = {
     "qsa_mqa_prefill_topk": (C.c_int, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f32, _i32,
                                        _i32, _vp, _i64, _vp, _sz, _vp]),
     "qsa_prefill_topk_workspace_size": (_sz, [_i64, _i32]),
+    "qsa_mqa_prefill_topk_noalloc": (C.c_int, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f32, _i32,
+                                               _i32, _vp, _i64, _vp]),
 }
 
 STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_ALIGNMENT", 3: "QSA_ERR_UNSUPPORTED",
@@ -213,4 +215,23 @@ def mqa_prefill_topk(q: torch.Tensor, k: torch.Tensor, ks: torch.Tensor, ke: tor
         _ptr(q), q.stride(0), q.stride(1), _ptr(k), k.stride(0), k.shape[0], _ptr(ks), _ptr(ke), T, scale, W,
         topk_k, _ptr(idx), idx.stride(0), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
+    return idx
+
+
+def mqa_prefill_topk_noalloc(q: torch.Tensor, k: torch.Tensor, ks: torch.Tensor, ke: torch.Tensor, W: int,
+                             topk_k: int, scale: float = SCALE, idx: torch.Tensor | None = None,
+                             stream=None) -> torch.Tensor:
+    """Prefill scores followed by per-row top-k through the library's static
+    scratch (no device allocation by the library) -> idx int32 [T, topk_k].
+    Calls that overlap on the GPU share that scratch and must be serialised."""
+    _prefill_checks(q, k, ks, ke)
+    T = q.shape[0]
+    if idx is None:
+        idx = torch.empty((T, topk_k), dtype=torch.int32, device=q.device)
+    _need(idx, "idx", torch.int32, 2)
+    if idx.shape != (T, topk_k) or idx.stride(1) != 1:
+        raise ValueError("idx must be [T, topk_k] with unit column stride")
+    _check("qsa_mqa_prefill_topk_noalloc", lib().qsa_mqa_prefill_topk_noalloc(
+        _ptr(q), q.stride(0), q.stride(1), _ptr(k), k.stride(0), k.shape[0], _ptr(ks), _ptr(ke), T, scale, W,
+        topk_k, _ptr(idx), idx.stride(0), _stream(stream)))
     return idx

@@ -293,6 +293,15 @@ qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream, float* pred_sta
   return launch_status("top-k kernel");
 }
 
+// Scratch of qsa_mqa_prefill_topk_noalloc: a fixed array that every GPU
+// loading this library holds until the process exits.  Host code must not
+// hand the symbol itself to a kernel (on the host it only stands in for the
+// device array); its device address is fetched once per device below.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
 }  // namespace
 
 // ================================================================ C ABI
@@ -432,6 +441,39 @@ qsa_status_t qsa_topk(const float* scores, int64_t score_stride, const int32_t* 
   if (st != QSA_OK) return st;
   if (rows == 0) return ok();
   return launch_topk(a, static_cast<cudaStream_t>(stream));
+}
+
+qsa_status_t qsa_mqa_prefill_topk_noalloc(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
+                                          int64_t k_stride, int64_t Nk, const int32_t* ks, const int32_t* ke,
+                                          int64_t T, float scale, int32_t W, int32_t topk_k, int32_t* idx,
+                                          int64_t idx_stride, void* stream) {
+  if (T < 0 || W < 1) return fail(QSA_ERR_INVALID_ARG, "T must be non-negative and W positive");
+  // one chunk of min(T, 64) rows of scores plus the selection state must fit
+  const int64_t rows = std::min<int64_t>(T, 64);
+  if ((size_t)rows * (size_t)W * sizeof(float) + 4096 > kNoAllocScratchBytes)
+    return fail(QSA_ERR_WORKSPACE,
+                "W = %d needs %lld bytes of scratch for one chunk of %lld rows; the static scratch holds %zu", W,
+                (long long)((size_t)rows * (size_t)W * sizeof(float) + 4096), (long long)rows,
+                kNoAllocScratchBytes);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(QSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      // first call on this device (with it current): the device address of the array
+      e = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+      if (e != cudaSuccess) {
+        g_noalloc_ptr[dev] = nullptr;
+        return fail(QSA_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
+      }
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return qsa_mqa_prefill_topk(q, q_stride_t, q_stride_h, k, k_stride, Nk, ks, ke, T, scale, W, topk_k, idx,
+                              idx_stride, scratch, kNoAllocScratchBytes, stream);
 }
 
 size_t qsa_prefill_topk_workspace_size(int64_t T, int32_t W) {

@@ -358,7 +358,7 @@ def cpu_baseline(b, budget_s: float = 10.0) -> dict:
     while True:
         b.oracle_step(threads)
         n += 1
-        if time.perf_counter() - t0 >= budget_s or n >= 50:
+        if time.perf_counter() - t0 >= budget_s or n >= 100000:
             break
     per_sample = (time.perf_counter() - t0) / n
     per_step = per_sample / frac

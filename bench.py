@@ -274,18 +274,27 @@ def make_bench(cfg: int, dev, seed: int):
 # ------------------------------------------------------------------ timing
 
 def sync_all(world: int):
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Largest value over the ranks (step times are reported as the slowest rank's)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_step: float, seconds_per_step: float, world: int, scale: float) -> float:
+    """Whole-job throughput: every rank processes its own batch of `units_per_step`."""
+    return units_per_step * world / seconds_per_step / scale
 
 
 def time_graph(b, steps: int, world: int, soak_s: float = 0.0, sampler: ClockSampler | None = None):

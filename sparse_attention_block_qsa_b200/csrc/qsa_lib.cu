@@ -79,6 +79,24 @@ qsa_status_t encode_bf16_map(CUtensorMap* map, int rank, void* base, const cuuin
   return QSA_OK;
 }
 
+// Store map of a W x rows fp32 matrix with the given row stride (elements),
+// box 32 x 16.  Returns false when TMA cannot address it (the caller then
+// stores element by element): the base and the row pitch must be multiples
+// of 16 bytes.
+bool encode_f32_store_map(CUtensorMap* map, float* base, int64_t W, int64_t rows, int64_t stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !aligned(base, 16) || W <= 0 || rows <= 0 || W > UINT32_MAX || rows > UINT32_MAX) return false;
+  const int64_t pitch = rows > 1 ? stride * 4 : ((W * 4 + 15) / 16) * 16;
+  if (pitch % 16 != 0 || pitch < W * 4 || pitch >= (int64_t(1) << 40)) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)W, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)pitch};
+  cuuint32_t box[2] = {32, (cuuint32_t)qsa::prefill::EPI_TOKENS};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------- device info
 struct DeviceInfo {
   int sms = 0;
@@ -227,8 +245,11 @@ qsa_status_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     p.out = a.out + r0 * a.out_stride;
     p.out_stride = a.out_stride;
     p.W = a.W;
-    qsa::prefill::prefill_kernel<<<sms, qsa::prefill::NUM_THREADS, qsa::prefill::SMEM_BYTES, stream>>>(tm_q, tm_k,
-                                                                                                      p);
+    CUtensorMap tm_out;
+    memset(&tm_out, 0, sizeof tm_out);
+    p.store_map = encode_f32_store_map(&tm_out, p.out, a.W, p.T, a.out_stride) ? 1 : 0;
+    qsa::prefill::prefill_kernel<<<sms, qsa::prefill::NUM_THREADS, qsa::prefill::SMEM_BYTES, stream>>>(
+        tm_q, tm_k, tm_out, p);
     st = launch_status("prefill kernel");
     if (st != QSA_OK) return st;
   }

@@ -129,6 +129,25 @@ __device__ __forceinline__ void tma_load_4d(void* dst, uint64_t* bar, const CUte
       : "memory");
 }
 
+// 2-D tiled store from shared memory, tracked by this thread's bulk group.
+// The coordinates must not be negative; parts of the box outside the tensor
+// are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_addr(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until every committed bulk store of this thread has finished reading
+// its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Wait until every committed bulk store of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------------ tcgen05
 
 // Allocate ncols TMEM columns (power of two >= 32); the base address is
@@ -176,6 +195,32 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// One K = 128 step of a bf16 product as eight K = 16 MMAs into d, the first
+// overwriting d.  a and b are the descriptors of the first 16-column slice of
+// the two K-major, 128-byte-swizzled operands; each holds its K columns in two
+// 64-column halves A_HALF and B_HALF bytes apart (in descriptor units of 16
+// bytes), and a 16-column step is 32 bytes.  The descriptors are plain sums
+// because shared-memory addresses stay below 256 KB.
+template <uint32_t A_HALF, uint32_t B_HALF>
+__device__ __forceinline__ void umma_bf16_k128(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t"
+      "setp.ne.b32 p0, %1, %1;\n\t"
+      "setp.eq.b32 p1, %1, %1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %10, %1, p0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %11, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %12, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %13, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %14, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %15, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %1, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %9, %17, %1, p1;\n\t}" ::"r"(d),
+      "r"(idesc), "l"(a), "l"(a + 2), "l"(a + 4), "l"(a + 6), "l"(a + A_HALF), "l"(a + A_HALF + 2),
+      "l"(a + A_HALF + 4), "l"(a + A_HALF + 6), "l"(b), "l"(b + 2), "l"(b + 4), "l"(b + 6), "l"(b + B_HALF),
+      "l"(b + B_HALF + 2), "l"(b + B_HALF + 4), "l"(b + B_HALF + 6)
+      : "memory");
+}
+
 // Arrive on *bar once all previously issued tcgen05 operations of this
 // thread have completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -219,6 +264,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 // scale * sum of the ReLU of four head dot products.
 __device__ __forceinline__ float head_sum_relu(float a, float b, float c, float d, float scale) {
   return scale * ((fmaxf(a, 0.f) + fmaxf(b, 0.f)) + (fmaxf(c, 0.f) + fmaxf(d, 0.f)));
+}
+
+// The same sum with one packed fp32x2 add: (a + c, b + d), then one add.
+__device__ __forceinline__ float head_sum_relu_x2(float a, float b, float c, float d, float scale) {
+  float x, y;
+  asm("{\n\t.reg .b64 p, q, r;\n\t"
+      "mov.b64 p, {%2, %3};\n\t"
+      "mov.b64 q, {%4, %5};\n\t"
+      "add.rn.f32x2 r, p, q;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(x), "=f"(y)
+      : "f"(fmaxf(a, 0.f)), "f"(fmaxf(b, 0.f)), "f"(fmaxf(c, 0.f)), "f"(fmaxf(d, 0.f)));
+  return (x + y) * scale;
 }
 
 }  // namespace qsa

@@ -6,10 +6,16 @@
 // score.  The design keeps as many key bytes in flight as the SM allows and
 // touches no shared memory on the way:
 //  * Work = the concatenation over requests of 8-key tiles (a tile never
-//    straddles a page: page sizes are multiples of 8).  Every warp of the
-//    grid takes an equal contiguous share of that list, so skewed context
-//    lengths cost nothing extra and no combine step is needed (each score is
-//    independent).
+//    straddles a page: page sizes are multiples of 8).  With more warps than
+//    requests, each request is cut into chunks of at most C tiles, C the
+//    smallest size for which all chunks fit the grid, and each warp takes one
+//    chunk, so skewed context lengths cost nothing extra and no warp pays a
+//    second query load; otherwise warps take equal contiguous shares of the
+//    tile list.  No combine step is needed (each score is independent).
+//  * The kernel is latency-bound for short batches, so the dependent memory
+//    round trips are kept to three (lengths, page entries with queries,
+//    keys): page-table rows and queries are prefetched into L2 while the
+//    lengths load, and the query and page-entry loads are issued together.
 //  * Each lane streams its part of the keys with 16-byte non-caching global
 //    loads straight into registers (4 tiles = 256 bytes per lane in flight),
 //    in the operand layout of mma.sync.m16n8k16 (B = 16 features x 8 keys).
@@ -36,7 +42,7 @@ constexpr int BATCH = 4;                // tiles in flight per warp
 constexpr int WARPS = 16;
 constexpr int NUM_THREADS = WARPS * 32;
 constexpr int MAX_B = 8192;             // requests per launch (prefix in shared memory)
-constexpr int FILL_BLOCK = 1024;        // columns per tail-fill block
+constexpr int64_t PREFETCH_MAX_LINES = 1 << 16;  // L2 prefetch budget (8 MB) for page tables and queries
 
 struct Params {
   const uint16_t* q;        // bf16 bits
@@ -56,6 +62,12 @@ struct Params {
   int64_t out_sb;
   int64_t out_st;
   int32_t W;
+  // L2 prefetch plan, set by the host: pf_rows page-table rows of
+  // pf_row_lines 128-byte lines each, then pf_q_lines query lines (3 per
+  // 256-byte query row); zero to skip
+  int32_t pf_row_lines;
+  int32_t pf_pt_lines;
+  int32_t pf_q_lines;
 };
 
 constexpr size_t SMEM_BYTES = sizeof(int32_t) * (MAX_B + 1);
@@ -101,20 +113,17 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint
 __device__ __forceinline__ void load_queries(const Params& p, int b, int lane, uint32_t (&a)[8][4]) {
   const int g = lane >> 2, c = lane & 3;
   const int t = g & 3, h = g >> 2;  // rows g and g + 8: heads h and h + 2 of token t
+  // Rows of tokens t >= Q read token Q - 1 instead (no branch, so the loads
+  // stay in flight); their scores are never stored.
   uint32_t w0[16], w1[16];
-  if (t < p.Q) {
-    const uint16_t* r0 = p.q + b * p.q_sb + t * p.q_st + h * p.q_sh;
-    const uint16_t* r1 = r0 + 2 * p.q_sh;
+  const uint16_t* r0 = p.q + b * p.q_sb + min(t, p.Q - 1) * p.q_st + h * p.q_sh;
+  const uint16_t* r1 = r0 + 2 * p.q_sh;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 x = __ldg(reinterpret_cast<const uint4*>(r0 + 8 * (c + 4 * i)));
-      const uint4 y = __ldg(reinterpret_cast<const uint4*>(r1 + 8 * (c + 4 * i)));
-      w0[4 * i] = x.x; w0[4 * i + 1] = x.y; w0[4 * i + 2] = x.z; w0[4 * i + 3] = x.w;
-      w1[4 * i] = y.x; w1[4 * i + 1] = y.y; w1[4 * i + 2] = y.z; w1[4 * i + 3] = y.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) w0[i] = w1[i] = 0u;
+  for (int i = 0; i < 4; ++i) {
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(r0 + 8 * (c + 4 * i)));
+    const uint4 y = __ldg(reinterpret_cast<const uint4*>(r1 + 8 * (c + 4 * i)));
+    w0[4 * i] = x.x; w0[4 * i + 1] = x.y; w0[4 * i + 2] = x.z; w0[4 * i + 3] = x.w;
+    w1[4 * i] = y.x; w1[4 * i + 1] = y.y; w1[4 * i + 2] = y.z; w1[4 * i + 3] = y.w;
   }
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
@@ -129,13 +138,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   extern __shared__ int32_t prefix[];  // prefix[b]: tiles before request b
   __shared__ uint32_t red[WARPS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gw = blockIdx.x * WARPS + warp;
+  const int nw = gridDim.x * WARPS;
+
+  // ---- the lengths load goes out first; the L2 prefetch of the page-table
+  // rows and queries is issued while it is in flight
+  const int len0 = tid < p.B ? __ldg(p.seq_lens + tid) : 0;
+  {
+    const int gt = blockIdx.x * NUM_THREADS + tid, nt = gridDim.x * NUM_THREADS;
+    // every prefetched address lies inside a page-table row's first
+    // max_pages entries or inside a 256-byte query row
+    for (int i = gt; i < p.pf_pt_lines; i += nt) {
+      const int b = i / p.pf_row_lines, l = i - b * p.pf_row_lines;
+      const char* row = reinterpret_cast<const char*>(p.page_table + (int64_t)b * p.pt_stride);
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(row + min(l * 128, p.max_pages * 4 - 1)));
+    }
+    for (int i = gt; i < p.pf_q_lines; i += nt) {
+      const int r = i / 3, l = i - r * 3;
+      const int b = r / (p.Q * 4), th = r - b * (p.Q * 4);
+      const char* row =
+          reinterpret_cast<const char*>(p.q + (int64_t)b * p.q_sb + (th >> 2) * p.q_st + (th & 3) * p.q_sh);
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(row + min(l * 128, 255)));
+    }
+  }
 
   // ---- tiles per request and their exclusive prefix (block-wide chunks)
   uint32_t carry = 0;
   for (int base = 0; base < p.B; base += NUM_THREADS) {
     const int b = base + tid;
     uint32_t v = 0;
-    if (b < p.B) v = (uint32_t)((scored_keys(p, __ldg(p.seq_lens + b)) + TILE - 1) / TILE);
+    if (b < p.B) v = (uint32_t)((scored_keys(p, base == 0 ? len0 : __ldg(p.seq_lens + b)) + TILE - 1) / TILE);
     uint32_t x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -158,30 +190,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   __syncthreads();
   const uint32_t total = carry;
 
-  const int64_t gw = (int64_t)blockIdx.x * WARPS + warp;
-  const int64_t nw = (int64_t)gridDim.x * WARPS;
-
-  // ---- -inf for the columns past each request's last tile
-  {
-    const int blocks_per_row = (p.W + FILL_BLOCK - 1) / FILL_BLOCK;
-    const int64_t nblocks = (int64_t)p.B * p.Q * blocks_per_row;
-    for (int64_t f = gw; f < nblocks; f += nw) {
-      const int64_t r = f / blocks_per_row;
-      const int b = (int)(r / p.Q), t = (int)(r % p.Q);
-      const int col0 = (int)(f % blocks_per_row) * FILL_BLOCK;
-      const int cov = (prefix[b + 1] - prefix[b]) * TILE;
-      const int lo = max(cov, col0), hi = min(col0 + FILL_BLOCK, p.W);
-      float* row = p.out + (int64_t)b * p.out_sb + (int64_t)t * p.out_st;
-      for (int n = lo + lane; n < hi; n += 32) row[n] = -INFINITY;
+  // ---- -inf for the columns past each request's last tile, written after
+  // the warp's tiles so that it stays off the path to the first key loads.
+  // With fewer rows than warps, a row's uncovered columns are striped over
+  // nw / rows warps in 32-column steps; otherwise each warp takes whole rows.
+  auto fill_tail = [&]() {
+    const int64_t rows = (int64_t)p.B * p.Q;
+    if (rows <= nw) {
+      const int r = gw % (int)rows, k0 = gw / (int)rows, ks = nw / (int)rows;
+      if (k0 < ks) {
+        const int b = r / p.Q, t = r - b * p.Q;
+        const int cov = (prefix[b + 1] - prefix[b]) * TILE;
+        float* row = p.out + (int64_t)b * p.out_sb + (int64_t)t * p.out_st;
+        for (int n = cov + k0 * 32 + lane; n < p.W; n += ks * 32) row[n] = -INFINITY;
+      }
+    } else {
+      for (int64_t r = gw; r < rows; r += nw) {
+        const int b = (int)(r / p.Q), t = (int)(r % p.Q);
+        const int cov = (prefix[b + 1] - prefix[b]) * TILE;
+        float* row = p.out + (int64_t)b * p.out_sb + (int64_t)t * p.out_st;
+        for (int n = cov + lane; n < p.W; n += 32) row[n] = -INFINITY;
+      }
     }
-  }
+  };
 
   // ---- this warp's share of the tiles
-  const uint32_t t_begin = (uint32_t)((uint64_t)gw * total / nw);
-  const uint32_t t_end = (uint32_t)((uint64_t)(gw + 1) * total / nw);
-  if (t_begin >= t_end) return;
+  uint32_t t_begin, t_end;
   int b;
-  {
+  if (2 * p.B <= nw) {
+    // chunks of at most C tiles that never cross a request: C is the least
+    // size with sum_b ceil(n_b / C) <= nw; ceil(total / (nw - B)) always fits
+    // and is within one of it.
+    uint32_t C = max((total + (uint32_t)(nw - p.B) - 1) / (uint32_t)(nw - p.B), 1u);
+    // warp index -> (request, chunk): walk the requests with one lane each
+    // and a running chunk count (requests are few when this branch runs)
+    int found = -1;
+    uint32_t chunk0 = 0, w_before = 0;
+    for (int base = 0; base < p.B && found < 0; base += 32) {
+      const int rb = base + lane;
+      const uint32_t nb = rb < p.B ? (uint32_t)(prefix[rb + 1] - prefix[rb]) : 0u;
+      const uint32_t wb = (nb + C - 1) / C;
+      uint32_t x = wb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      const uint32_t excl = w_before + x - wb;
+      const bool mine = rb < p.B && (uint32_t)gw >= excl && (uint32_t)gw < excl + wb;
+      const unsigned m = __ballot_sync(0xffffffffu, mine);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        found = base + src;
+        chunk0 = (uint32_t)gw - __shfl_sync(0xffffffffu, excl, src);
+      }
+      w_before += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (found < 0) {
+      fill_tail();
+      return;
+    }
+    b = found;
+    const uint32_t nb = (uint32_t)(prefix[b + 1] - prefix[b]);
+    t_begin = (uint32_t)prefix[b] + chunk0 * C;
+    t_end = (uint32_t)prefix[b] + min((chunk0 + 1) * C, nb);
+    if (t_begin >= t_end) {
+      fill_tail();
+      return;
+    }
+  } else {
+    const uint32_t per = total / (uint32_t)nw, rem = total % (uint32_t)nw;
+    t_begin = (uint32_t)gw * per + min((uint32_t)gw, rem);
+    t_end = t_begin + per + ((uint32_t)gw < rem ? 1u : 0u);
+    if (t_begin >= t_end) {
+      fill_tail();
+      return;
+    }
     int lo = 0, hi = p.B - 1;  // last request with prefix[b] <= t_begin
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -207,16 +291,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   // that no page-table load sits between two batches of key loads.
   int j0 = j;
   int entry = -1;
+  // The raw entry stays a pending load until a batch reads it; the range
+  // check happens there.
   auto fetch_entries = [&]() {
-    entry = -1;
-    const int tile = j0 + lane;
-    if (tile < nt_b) {
-      const int logical = (tile * TILE) >> p.log2_ps;
-      if (logical < p.max_pages) {
-        const int e = __ldg(p.page_table + (int64_t)b * p.pt_stride + logical);
-        if (e >= 0 && (int64_t)e < p.num_pages) entry = e;
-      }
-    }
+    const int tile = min(j0 + lane, nt_b - 1);
+    const int logical = min((tile * TILE) >> p.log2_ps, p.max_pages - 1);
+    entry = p.max_pages > 0 ? __ldg(p.page_table + (int64_t)b * p.pt_stride + logical) : -1;
   };
   fetch_entries();
 
@@ -227,6 +307,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
 #pragma unroll
     for (int u = 0; u < BATCH; ++u) {
       ent[u] = __shfl_sync(0xffffffffu, entry, (j - j0 + u) & 31);
+      // tiles past the request's pages (logical page >= max_pages) and
+      // entries outside the pool are invalid
+      const bool in_table = (((j + u) * TILE) >> p.log2_ps) < p.max_pages;
+      if (!(in_table && ent[u] >= 0 && (int64_t)ent[u] < p.num_pages)) ent[u] = -1;
       if (u < cnt && ent[u] >= 0) {
         const int row = ((j + u) * TILE + g) & ps_mask;
         const uint16_t* kr = p.k_cache + (int64_t)ent[u] * p.k_page_stride + (int64_t)row * p.k_row_stride;
@@ -290,6 +374,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
       load_queries(p, b, lane, qa);
     }
   }
+  fill_tail();
 }
 
 }  // namespace decode

@@ -7,15 +7,15 @@
 // touches no shared memory on the way:
 //  * Work = the concatenation over requests of 8-key tiles (a tile never
 //    straddles a page: page sizes are multiples of 8).  With more warps than
-//    requests, each request is cut into chunks of at most C tiles, C the
+//    requests (and more than one request), each request is cut into chunks of at most C tiles, C the
 //    smallest size for which all chunks fit the grid, and each warp takes one
 //    chunk, so skewed context lengths cost nothing extra and no warp pays a
 //    second query load; otherwise warps take equal contiguous shares of the
 //    tile list.  No combine step is needed (each score is independent).
 //  * The kernel is latency-bound for short batches, so the dependent memory
 //    round trips are kept to three (lengths, page entries with queries,
-//    keys): page-table rows and queries are prefetched into L2 while the
-//    lengths load, and the query and page-entry loads are issued together.
+//    keys): the lengths load is the first instruction, and the query and
+//    page-entry loads are issued together.
 //  * Each lane streams its part of the keys with 16-byte non-caching global
 //    loads straight into registers (4 tiles = 256 bytes per lane in flight),
 //    in the operand layout of mma.sync.m16n8k16 (B = 16 features x 8 keys).
@@ -42,7 +42,6 @@ constexpr int BATCH = 4;                // tiles in flight per warp
 constexpr int WARPS = 16;
 constexpr int NUM_THREADS = WARPS * 32;
 constexpr int MAX_B = 8192;             // requests per launch (prefix in shared memory)
-constexpr int64_t PREFETCH_MAX_LINES = 1 << 16;  // L2 prefetch budget (8 MB) for page tables and queries
 
 struct Params {
   const uint16_t* q;        // bf16 bits
@@ -62,12 +61,6 @@ struct Params {
   int64_t out_sb;
   int64_t out_st;
   int32_t W;
-  // L2 prefetch plan, set by the host: pf_rows page-table rows of
-  // pf_row_lines 128-byte lines each, then pf_q_lines query lines (3 per
-  // 256-byte query row); zero to skip
-  int32_t pf_row_lines;
-  int32_t pf_pt_lines;
-  int32_t pf_q_lines;
 };
 
 constexpr size_t SMEM_BYTES = sizeof(int32_t) * (MAX_B + 1);
@@ -141,26 +134,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   const int gw = blockIdx.x * WARPS + warp;
   const int nw = gridDim.x * WARPS;
 
-  // ---- the lengths load goes out first; the L2 prefetch of the page-table
-  // rows and queries is issued while it is in flight
+  // ---- the lengths load goes out first
   const int len0 = tid < p.B ? __ldg(p.seq_lens + tid) : 0;
-  {
-    const int gt = blockIdx.x * NUM_THREADS + tid, nt = gridDim.x * NUM_THREADS;
-    // every prefetched address lies inside a page-table row's first
-    // max_pages entries or inside a 256-byte query row
-    for (int i = gt; i < p.pf_pt_lines; i += nt) {
-      const int b = i / p.pf_row_lines, l = i - b * p.pf_row_lines;
-      const char* row = reinterpret_cast<const char*>(p.page_table + (int64_t)b * p.pt_stride);
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(row + min(l * 128, p.max_pages * 4 - 1)));
-    }
-    for (int i = gt; i < p.pf_q_lines; i += nt) {
-      const int r = i / 3, l = i - r * 3;
-      const int b = r / (p.Q * 4), th = r - b * (p.Q * 4);
-      const char* row =
-          reinterpret_cast<const char*>(p.q + (int64_t)b * p.q_sb + (th >> 2) * p.q_st + (th & 3) * p.q_sh);
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(row + min(l * 128, 255)));
-    }
-  }
 
   // ---- tiles per request and their exclusive prefix (block-wide chunks)
   uint32_t carry = 0;
@@ -217,7 +192,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   // ---- this warp's share of the tiles
   uint32_t t_begin, t_end;
   int b;
-  if (2 * p.B <= nw) {
+  if (p.B > 1 && 2 * p.B <= nw) {
     // chunks of at most C tiles that never cross a request: C is the least
     // size with sum_b ceil(n_b / C) <= nw; ceil(total / (nw - B)) always fits
     // and is within one of it.

@@ -422,16 +422,6 @@ qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_
     p.page_table = max_pages > 0 ? page_table + (int64_t)b0 * pt_stride : page_table;
     p.seq_lens = seq_lens + b0;
     p.out = out + (int64_t)b0 * out_stride_b;
-    {
-      // L2 prefetch plan: page-table rows (any alignment: one extra line) and
-      // query rows, within a fixed line budget
-      const int64_t row_lines = max_pages > 0 ? ((int64_t)max_pages * 4 + 127) / 128 + 1 : 0;
-      const int64_t pt_lines = (int64_t)p.B * row_lines, q_lines = (int64_t)p.B * Q * 4 * 3;
-      const bool on = pt_lines + q_lines <= qsa::decode::PREFETCH_MAX_LINES;
-      p.pf_row_lines = on ? (int32_t)row_lines : 0;
-      p.pf_pt_lines = on ? (int32_t)pt_lines : 0;
-      p.pf_q_lines = on ? (int32_t)q_lines : 0;
-    }
     qsa::decode::decode_kernel<<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES,
                                  static_cast<cudaStream_t>(stream)>>>(p);
     st = launch_status("decode kernel");

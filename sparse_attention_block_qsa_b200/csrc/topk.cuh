@@ -4,11 +4,13 @@
 //
 // Persistent CTAs, each over a contiguous range of rows (neighbouring query
 // rows score alike).  Two kernels share the selection logic:
-//  * topk_stream_kernel (rows 16-byte aligned, W a multiple of 4), two CTAs
-//    per SM: a producer warp streams every row of the CTA's range as 16 KB
-//    bulk copies into a 4-slot shared-memory ring without pausing between
-//    rows; 8 selecting warps read the ring.  While one CTA resolves a row,
-//    the other keeps streaming.
+//  * topk_stream_kernel (rows 16-byte aligned, W a multiple of 4), three
+//    CTAs per SM: a producer warp streams every row of the CTA's range as
+//    16 KB bulk copies into a 2-slot shared-memory ring without pausing
+//    between rows; 8 selecting warps read the ring.  The selection work is
+//    latency-bound (short phases between barriers), so the SM holds as many
+//    CTAs as registers allow (72 per thread) and while one CTA resolves a
+//    row the others keep streaming.
 //  * topk_rows_kernel (any alignment): 8 warps read each row with batched
 //    loads themselves.
 // Per row:
@@ -41,7 +43,7 @@ namespace topk {
 constexpr int THREADS = 256;          // selecting threads (both kernels)
 constexpr int NWARPS = THREADS / 32;
 constexpr int ROWS_CTAS_PER_SM = 4;
-constexpr int STREAM_CTAS_PER_SM = 2;
+constexpr int STREAM_CTAS_PER_SM = 3;
 constexpr int HBITS = 11;
 constexpr int HBINS = 1 << HBITS;
 constexpr int HSHIFT = 32 - HBITS;
@@ -54,7 +56,7 @@ constexpr int FBINS = 2048;           // fast-path histogram
 constexpr uint32_t ZERO_KEY = 0x80000000u;
 constexpr float PREDICT_MARGIN = 0.9f;
 constexpr int CHUNK = 4096;           // floats per ring slot (16 KB)
-constexpr int NST = 4;                // ring slots
+constexpr int NST = 2;                // ring slots
 constexpr int STREAM_THREADS = THREADS + 32;
 static_assert(FBINS == HBINS, "the fast path and the exact path share one histogram");
 
@@ -152,14 +154,14 @@ __device__ __forceinline__ void block_scan2(uint32_t& a, uint32_t& b, uint32_t* 
 // Visit every column j < len of a row in global memory with its score; all
 // selecting threads take every step together (columns past len arrive as
 // -inf), so f may use warp-collective operations.  Loads are issued in
-// batches of 8 x 16 bytes.
+// batches of 4 x 16 bytes per thread.
 template <typename F>
 __device__ __forceinline__ void for_each_score(const Params& p, const float* row, int len, F&& f) {
   const int tid = threadIdx.x;
   if (p.vec4) {
     const float4* row4 = reinterpret_cast<const float4*>(row);
     const int n4 = (len + 3) >> 2;
-    constexpr int U = 8;
+    constexpr int U = 4;
     for (int i0 = 0; i0 < n4; i0 += U * THREADS) {
       float4 x[U];
 #pragma unroll

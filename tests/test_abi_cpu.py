@@ -126,7 +126,12 @@ def test_fused_rejects_small_workspace():
     st = L.qsa_mqa_prefill_topk(A, 512, 128, A + S, 128, 1000, A + 2 * S, A + 3 * S, 1000, 0.088, 1000, 512,
                                 A + 4 * S, 512, A + 5 * S, 63 * 1000 * 4, None)
     assert st == WS, L.qsa_last_error_detail().decode()
-    assert L.qsa_prefill_topk_workspace_size(16384, 26624) == 16384 * 26624 * 4 + 4096
+    # one chunk of all rows in either layout: at least the score-row layout's
+    # T rows of W floats plus 4096 bytes, growing with T, zero when empty
+    size = L.qsa_prefill_topk_workspace_size
+    assert size(16384, 26624) >= 16384 * 26624 * 4 + 4096
+    assert size(64, 26624) < size(65, 26624) < size(16384, 26624)
+    assert size(0, 26624) == 0 and size(16, 0) == 0
 
 
 def test_binding_refuses_cpu_tensors():

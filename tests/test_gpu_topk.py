@@ -79,7 +79,7 @@ def test_fused_prefill_topk_matches_separate_calls():
     scores = qsa.mqa_prefill(q, k, ks_d, ke_d, p.W)
     want = qsa.topk(scores, 512)
     for rows_in_ws in (p.T, 64, 128, 200):
-        ws = torch.empty(rows_in_ws * p.W + 1024, dtype=torch.float32, device=DEV)
+        ws = torch.empty(qsa.prefill_topk_workspace_size(rows_in_ws, p.W) // 4 + 1, dtype=torch.float32, device=DEV)
         got = qsa.mqa_prefill_topk(q, k, ks_d, ke_d, p.W, 512, ws)
         assert torch.equal(got, want), rows_in_ws
     torch.cuda.synchronize()
@@ -106,3 +106,32 @@ def test_fused_prefill_topk_full_config_sampled():
     loose, _ = prefill_bounds(p.q, p.k, ks, p.W, SCALE, rows=rows)
     for i, r in enumerate(rows):
         topk_sets_agree(idx[r], ora_idx[i], ref[i], loose[i], wl.TOPK_K)
+
+
+def _fused_vs_separate(p, q, k, k_top=512):
+    ks, ke = oracle.prefill_intervals(p.cu_seqlens_q, p.seq_lens, p.key_offsets)
+    ks_d, ke_d = torch.from_numpy(ks).to(DEV), torch.from_numpy(ke).to(DEV)
+    q, k = q.to(DEV), k.to(DEV)
+    want = qsa.topk(qsa.mqa_prefill(q, k, ks_d, ke_d, p.W), k_top)
+    ws = torch.empty(qsa.prefill_topk_workspace_size(p.T, p.W) // 4 + 1, dtype=torch.float32, device=DEV)
+    got = qsa.mqa_prefill_topk(q, k, ks_d, ke_d, p.W, k_top, ws)
+    torch.cuda.synchronize()
+    assert qsa.device_error() == 0
+    assert torch.equal(got, want)
+
+
+@pytest.mark.parametrize("sampled_high", [True, False])
+def test_fused_prefill_topk_ties_and_skew(sampled_high):
+    """Every 16th key scores far above all others (about 190 equal scores
+    inside the top 512 of a row) or exactly zero (a block of ties at the
+    bottom): the fused entry must still equal top-k over the separate scores,
+    ties resolved to the lower column."""
+    p = wl.make_prefill("fused_fallback", [96, 70], [12000, 9000], seed=6)
+    q = torch.zeros_like(p.q)
+    q[:, :, 0] = 1.0
+    k = torch.randn(p.k.shape, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16) * 0.1
+    k[:, 0] = k[:, 0].abs() + 0.5
+    sampled = torch.arange(p.Nk) % 16 == 0
+    k[sampled, 0] = 8.0 if sampled_high else 0.0
+    k[sampled, 1:] = 0.0
+    _fused_vs_separate(p, q, k)

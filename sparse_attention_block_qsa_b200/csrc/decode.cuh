@@ -134,11 +134,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   const int gw = blockIdx.x * WARPS + warp;
   const int nw = gridDim.x * WARPS;
 
-  // ---- the lengths load goes out first
-  const int len0 = tid < p.B ? __ldg(p.seq_lens + tid) : 0;
+  // ---- the lengths load goes out first.  With at most 32 requests every
+  // warp builds the request plan in its own registers (lane b: request b), so
+  // no warp waits for another; otherwise one block-wide scan in shared memory.
+  const bool warp_plan = p.B <= 32;
+  const int len0 = warp_plan ? (lane < p.B ? __ldg(p.seq_lens + lane) : 0) : (tid < p.B ? __ldg(p.seq_lens + tid) : 0);
+  uint32_t total = 0, lp = 0;   // warp plan: lp = tiles before request `lane` (all tiles for lanes >= B)
+  if (warp_plan) {
+    const uint32_t v = lane < p.B ? (uint32_t)((scored_keys(p, len0) + TILE - 1) / TILE) : 0u;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    lp = x - v;
+    total = __shfl_sync(0xffffffffu, x, 31);
+  }
+  // tiles before request b (b <= B); every lane of the warp calls it
+  auto pfx = [&](int b) -> uint32_t {
+    if (warp_plan) {
+      const uint32_t s = __shfl_sync(0xffffffffu, lp, b & 31);
+      return b < 32 ? s : total;
+    }
+    return (uint32_t)prefix[b];
+  };
 
   // ---- tiles per request and their exclusive prefix (block-wide chunks)
   uint32_t carry = 0;
+  if (!warp_plan) {
   for (int base = 0; base < p.B; base += NUM_THREADS) {
     const int b = base + tid;
     uint32_t v = 0;
@@ -163,7 +187,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   }
   if (tid == 0) prefix[p.B] = (int32_t)carry;
   __syncthreads();
-  const uint32_t total = carry;
+  total = carry;
+  }
 
   // ---- -inf for the columns past each request's last tile, written after
   // the warp's tiles so that it stays off the path to the first key loads.
@@ -175,14 +200,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
       const int r = gw % (int)rows, k0 = gw / (int)rows, ks = nw / (int)rows;
       if (k0 < ks) {
         const int b = r / p.Q, t = r - b * p.Q;
-        const int cov = (prefix[b + 1] - prefix[b]) * TILE;
+        const int cov = (int)(pfx(b + 1) - pfx(b)) * TILE;
         float* row = p.out + (int64_t)b * p.out_sb + (int64_t)t * p.out_st;
         for (int n = cov + k0 * 32 + lane; n < p.W; n += ks * 32) row[n] = -INFINITY;
       }
     } else {
       for (int64_t r = gw; r < rows; r += nw) {
         const int b = (int)(r / p.Q), t = (int)(r % p.Q);
-        const int cov = (prefix[b + 1] - prefix[b]) * TILE;
+        const int cov = (int)(pfx(b + 1) - pfx(b)) * TILE;
         float* row = p.out + (int64_t)b * p.out_sb + (int64_t)t * p.out_st;
         for (int n = cov + lane; n < p.W; n += 32) row[n] = -INFINITY;
       }
@@ -203,7 +228,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
     uint32_t chunk0 = 0, w_before = 0;
     for (int base = 0; base < p.B && found < 0; base += 32) {
       const int rb = base + lane;
-      const uint32_t nb = rb < p.B ? (uint32_t)(prefix[rb + 1] - prefix[rb]) : 0u;
+      // every lane calls pfx (a shuffle in the warp plan); rb + 1 <= B + 31
+      // stays inside the shared table, as this branch has 2B <= nw
+      const uint32_t p1 = pfx(rb + 1), p0 = pfx(rb);
+      const uint32_t nb = rb < p.B ? p1 - p0 : 0u;
       const uint32_t wb = (nb + C - 1) / C;
       uint32_t x = wb;
 #pragma unroll
@@ -226,9 +254,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
       return;
     }
     b = found;
-    const uint32_t nb = (uint32_t)(prefix[b + 1] - prefix[b]);
-    t_begin = (uint32_t)prefix[b] + chunk0 * C;
-    t_end = (uint32_t)prefix[b] + min((chunk0 + 1) * C, nb);
+    const uint32_t pb = pfx(b), nb = pfx(b + 1) - pb;
+    t_begin = pb + chunk0 * C;
+    t_end = pb + min((chunk0 + 1) * C, nb);
     if (t_begin >= t_end) {
       fill_tail();
       return;
@@ -244,13 +272,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
     int lo = 0, hi = p.B - 1;  // last request with prefix[b] <= t_begin
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if ((uint32_t)prefix[mid] <= t_begin) lo = mid;
+      if (pfx(mid) <= t_begin) lo = mid;
       else hi = mid - 1;
     }
     b = lo;
-    while ((uint32_t)prefix[b + 1] <= t_begin) ++b;  // skip requests without tiles
+    while (pfx(b + 1) <= t_begin) ++b;  // skip requests without tiles
   }
-  int j = (int)(t_begin - (uint32_t)prefix[b]);
+  int j = (int)(t_begin - pfx(b));
   uint32_t left = t_end - t_begin;
   int ob = b;
 
@@ -261,7 +289,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   uint32_t qa[8][4];
   load_queries(p, b, lane, qa);
   int L = __ldg(p.seq_lens + b);
-  int nt_b = prefix[b + 1] - prefix[b];
+  int nt_b = (int)(pfx(b + 1) - pfx(b));
   // Page of tile j0 + lane of the current request, read 32 tiles ahead so
   // that no page-table load sits between two batches of key loads.
   int j0 = j;
@@ -305,10 +333,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
       if (j == nt_b) {
         do {
           ++b;
-        } while (prefix[b + 1] == prefix[b]);
+        } while (pfx(b + 1) == pfx(b));
         j = 0;
         j0 = 0;
-        nt_b = prefix[b + 1] - prefix[b];
+        nt_b = (int)(pfx(b + 1) - pfx(b));
         fetch_entries();
       } else if (j - j0 == 32) {
         j0 = j;

@@ -69,6 +69,15 @@ const char* qsa_last_error_detail(void);
  * never for the hot path). */
 qsa_status_t qsa_device_error(uint32_t* bits);
 
+/* qsa_selftest_bounded_wait - a diagnostic of the failure handling above; the
+ * pages have no counterpart.  Launches one warp on `stream` whose first
+ * thread waits, with the same bounded wait the kernels use and a limit of
+ * timeout_ns (at most 10 s), on an mbarrier phase that nothing completes
+ * (arrive == 0) or that the thread completes itself first (arrive != 0).  A
+ * wait that runs out sets QSA_DEVERR_WAIT_TIMEOUT in the device error word and
+ * the kernel returns; the context stays usable.  For tests. */
+qsa_status_t qsa_selftest_bounded_wait(uint64_t timeout_ns, int32_t arrive, void* stream);
+
 /*
  * qsa_mqa_decode - decode and speculative-decode scores over a paged
  * compressed key cache.

@@ -6,7 +6,9 @@ intervals, per-row top-k selection and the fused prefill + top-k path.
 This package is the thin Python binding over that library.
 """
 from ._abi import (SCALE, QSAError, device_error, lib, mqa_decode, mqa_prefill, mqa_prefill_topk,
-                   mqa_prefill_topk_noalloc, prefill_intervals, prefill_topk_workspace_size, topk)
+                   mqa_prefill_topk_noalloc, prefill_intervals, prefill_topk_workspace_size,
+                   selftest_bounded_wait, topk)
 
 __all__ = ["SCALE", "QSAError", "device_error", "lib", "mqa_decode", "mqa_prefill", "mqa_prefill_topk",
-           "mqa_prefill_topk_noalloc", "prefill_intervals", "prefill_topk_workspace_size", "topk"]
+           "mqa_prefill_topk_noalloc", "prefill_intervals", "prefill_topk_workspace_size",
+           "selftest_bounded_wait", "topk"]

@@ -23,6 +23,7 @@ SIGNATURES = {
     "qsa_status_string": (C.c_char_p, [C.c_int]),
     "qsa_last_error_detail": (C.c_char_p, []),
     "qsa_device_error": (C.c_int, [C.POINTER(C.c_uint32)]),
+    "qsa_selftest_bounded_wait": (C.c_int, [C.c_uint64, _i32, _vp]),
     "qsa_mqa_decode": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _i64, _i32, _i64, _i64, _vp, _i64, _i32,
                                  _vp, _i32, _i32, _f32, _vp, _i64, _i64, _i32, _vp]),
     "qsa_mqa_prefill": (C.c_int, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f32, _vp, _i64,
@@ -93,6 +94,13 @@ def device_error() -> int:
     v = C.c_uint32(0)
     _check("qsa_device_error", lib().qsa_device_error(C.byref(v)))
     return v.value
+
+
+def selftest_bounded_wait(timeout_ns: int, arrive: bool, stream=None) -> None:
+    """Launch the bounded-wait diagnostic (a wait on a barrier phase that
+    nothing completes unless `arrive`); see qsa_selftest_bounded_wait."""
+    _check("qsa_selftest_bounded_wait", lib().qsa_selftest_bounded_wait(timeout_ns, 1 if arrive else 0,
+                                                                       _stream(stream)))
 
 
 def mqa_decode(q: torch.Tensor, k_cache: torch.Tensor, page_table: torch.Tensor, seq_lens: torch.Tensor,

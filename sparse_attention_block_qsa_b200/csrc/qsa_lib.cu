@@ -314,6 +314,18 @@ qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream, float* pred_sta
   return launch_status("top-k kernel");
 }
 
+// One thread waits on an mbarrier that nothing arrives on (unless `arrive`),
+// with the kernels' bounded wait and the given limit.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns, int32_t arrive) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    qsa::mbar_init(&bar, 1);
+    qsa::fence_mbar_init();
+    if (arrive) qsa::mbar_arrive(&bar);
+    if (!qsa::mbar_wait_for(&bar, 0, nullptr, timeout_ns)) qsa::record_device_error(QSA_DEVERR_WAIT_TIMEOUT);
+  }
+}
+
 // Scratch of qsa_mqa_prefill_topk_noalloc: a fixed array that every GPU
 // loading this library holds until the process exits.  Host code must not
 // hand the symbol itself to a kernel (on the host it only stands in for the
@@ -350,6 +362,15 @@ qsa_status_t qsa_device_error(uint32_t* bits) {
   if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
   *bits = v;
   return ok();
+}
+
+qsa_status_t qsa_selftest_bounded_wait(uint64_t timeout_ns, int32_t arrive, void* stream) {
+  if (timeout_ns > 10000000000ull) return fail(QSA_ERR_INVALID_ARG, "timeout_ns above 10 s");
+  int sms = 0;
+  qsa_status_t st = device_info(&sms);
+  if (st != QSA_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns, arrive);
+  return launch_status("self-test kernel");
 }
 
 qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,

@@ -65,17 +65,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false if
-// the wait ran past the time limit or if *abort became non-zero meanwhile.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// the wait ran past timeout_ns of global time or if *abort became non-zero
+// meanwhile.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t start = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (global_timer_ns() - start > QSA_WAIT_TIMEOUT_NS) return false;
+      if (global_timer_ns() - start > timeout_ns) return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, QSA_WAIT_TIMEOUT_NS);
 }
 
 // ------------------------------------------------------------------ fences
@@ -117,15 +123,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, uint64_t* bar, const CUte
       "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
       "[%2];" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_4d(void* dst, uint64_t* bar, const CUtensorMap* map, int32_t c0,
-                                            int32_t c1, int32_t c2, int32_t c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
-      "%6}], [%2];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 
@@ -185,16 +182,6 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(uint32_t M, uint32_t 
          | ((M >> 4) << 24);  // M / 16
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // One K = 128 step of a bf16 product as eight K = 16 MMAs into d, the first
 // overwriting d.  a and b are the descriptors of the first 16-column slice of
 // the two K-major, 128-byte-swizzled operands; each holds its K columns in two
@@ -231,20 +218,7 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 32 lanes x 32 bit, 16 consecutive columns: thread i gets lane (base + i).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// 32 lanes x 32 bit, 32 consecutive columns.
+// 32 lanes x 32 bit, 32 consecutive columns: thread i gets lane (base + i).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   uint32_t r[32];
   asm volatile(
@@ -261,12 +235,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 
 // ------------------------------------------------------------------ math
 
-// scale * sum of the ReLU of four head dot products.
-__device__ __forceinline__ float head_sum_relu(float a, float b, float c, float d, float scale) {
-  return scale * ((fmaxf(a, 0.f) + fmaxf(b, 0.f)) + (fmaxf(c, 0.f) + fmaxf(d, 0.f)));
-}
-
-// The same sum with one packed fp32x2 add: (a + c, b + d), then one add.
+// scale * sum of the ReLU of four head dot products, with one packed fp32x2
+// add: (relu(a) + relu(c), relu(b) + relu(d)), then one add and the scale.
 __device__ __forceinline__ float head_sum_relu_x2(float a, float b, float c, float d, float scale) {
   float x, y;
   asm("{\n\t.reg .b64 p, q, r;\n\t"

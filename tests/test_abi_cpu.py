@@ -139,3 +139,8 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(TypeError):
         qsa.mqa_decode(q, torch.zeros(1, 16, 1, 128, dtype=torch.bfloat16), torch.zeros(1, 1, dtype=torch.int32),
                        torch.zeros(1, dtype=torch.int32), 4)
+
+
+def test_selftest_rejects_long_limit():
+    L = qsa.lib()
+    assert L.qsa_selftest_bounded_wait(20_000_000_000, 0, None) == INVALID, L.qsa_last_error_detail().decode()

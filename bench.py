@@ -70,19 +70,30 @@ def read_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def source_hash() -> str:
+    """Digest of the kernel sources (every file of csrc/) with comments and
+    blank space removed, so that it changes exactly when the code does."""
+    import hashlib
+    import re
+    src = os.path.join(ROOT, "sparse_attention_block_qsa_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(src)):
+        with open(os.path.join(src, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(f.encode())
+        h.update(" ".join(text.split()).encode())
+    return h.hexdigest()[:12]
+
+
 def read_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel source."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.md")
     if not os.path.exists(path):
         return None
-    import hashlib
-    src = os.path.join(ROOT, "sparse_attention_block_qsa_b200", "csrc")
-    h = hashlib.sha256()
-    for f in sorted(os.listdir(src)):
-        with open(os.path.join(src, f), "rb") as fh:
-            h.update(fh.read())
-    sha = h.hexdigest()[:12]
+    sha = source_hash()
     for line in open(path):
         parts = [p.strip() for p in line.strip().strip("|").split("|")]
         if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload and parts[2] == sha:

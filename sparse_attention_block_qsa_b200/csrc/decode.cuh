@@ -6,16 +6,18 @@
 // score.  The design keeps as many key bytes in flight as the SM allows and
 // touches no shared memory on the way:
 //  * Work = the concatenation over requests of 8-key tiles (a tile never
-//    straddles a page: page sizes are multiples of 8).  With more warps than
-//    requests (and more than one request), each request is cut into chunks of at most C tiles, C the
-//    smallest size for which all chunks fit the grid, and each warp takes one
-//    chunk, so skewed context lengths cost nothing extra and no warp pays a
-//    second query load; otherwise warps take equal contiguous shares of the
-//    tile list.  No combine step is needed (each score is independent).
+//    straddles a page: page sizes are multiples of 8).  With more than one
+//    request and at least twice as many warps as requests, each request is
+//    cut into chunks of at most C tiles, C the smallest size for which all
+//    chunks fit the grid, and each warp takes one chunk, so skewed context
+//    lengths cost nothing extra and no warp pays a second query load;
+//    otherwise warps take equal contiguous shares of the tile list.  No
+//    combine step is needed (each score is independent).
 //  * The kernel is latency-bound for short batches, so the dependent memory
 //    round trips are kept to three (lengths, page entries with queries,
-//    keys): the lengths load is the first instruction, and the query and
-//    page-entry loads are issued together.
+//    keys): the lengths load is the first instruction, the query and
+//    page-entry loads are issued together, and with at most 32 requests each
+//    warp plans its work in registers, with no block barrier.
 //  * Each lane streams its part of the keys with 16-byte non-caching global
 //    loads straight into registers (4 tiles = 256 bytes per lane in flight),
 //    in the operand layout of mma.sync.m16n8k16 (B = 16 features x 8 keys).

@@ -1,5 +1,6 @@
-// sm_100a building blocks written as inline PTX: mbarriers, TMA tiled loads,
-// tcgen05 (TMEM allocation, UMMA issue, commit, TMEM loads) and bounded waits.
+// sm_100a building blocks written as inline PTX: mbarriers, TMA tiled loads
+// and stores with bulk groups, tcgen05 (TMEM allocation, UMMA issue, commit,
+// TMEM loads) and bounded waits.
 //
 // Every wait here is bounded: after QSA_WAIT_TIMEOUT_NS of global time it
 // gives up, so a kernel can record an error and leave instead of hanging.

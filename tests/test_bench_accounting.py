@@ -58,3 +58,20 @@ def test_prefill_flops_reproduce_printed_tflops():
 def test_job_throughput_counts_every_rank():
     assert bench.job_throughput(1e9, 1e-3, 1, 1e9) == 1000.0
     assert bench.job_throughput(1e9, 1e-3, 4, 1e9) == 4000.0
+
+
+def test_source_digest_ignores_comments_and_blank_space(tmp_path, monkeypatch):
+    """The DRAM-traffic rows are keyed by bench.source_hash(): a comment or
+    blank-space edit must keep the key, a code edit must change it."""
+    import shutil
+    root = tmp_path / "repo"
+    src = root / "sparse_attention_block_qsa_b200" / "csrc"
+    shutil.copytree(os.path.join(bench.ROOT, "sparse_attention_block_qsa_b200", "csrc"), src)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    base = bench.source_hash()
+    f = src / "decode.cuh"
+    text = f.read_text()
+    f.write_text(text.replace("#pragma once", "// a new comment\n/* and a block\n   comment */\n\n#pragma   once", 1))
+    assert bench.source_hash() == base
+    f.write_text(text.replace("constexpr int BATCH = 4;", "constexpr int BATCH = 2;", 1))
+    assert bench.source_hash() != base

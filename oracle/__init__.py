@@ -38,6 +38,10 @@ def _bind(L: C.CDLL) -> C.CDLL:
     L.qsa_oracle_prefill_entries.argtypes = [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _f64,
                                              _vp, _vp, _i64, _vp, _int]
     L.qsa_oracle_topk.argtypes = [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _int]
+    L.qsa_oracle_e4m3_to_double.argtypes = [C.c_uint8]
+    L.qsa_oracle_e4m3_to_double.restype = C.c_double
+    L.qsa_oracle_decode_fp8.argtypes = [_vp, _i64, _i64, _i64, _vp, _f64, _i64, _i64, _i64, _i64,
+                                        _vp, _i64, _i64, _vp, _i64, _i64, _f64, _vp, _i64, _int]
     return L
 
 
@@ -115,6 +119,37 @@ class Oracle:
                                  kb.shape[1], kst[0], kst[1], _ptr(pt), pt.shape[1],
                                  pt.shape[1], _ptr(sl), B, Q, float(scale), _ptr(out), W,
                                  threads)
+        return out
+
+    def e4m3_to_double(self, code: int) -> float:
+        """Value of one fp8 E4M3 code."""
+        return float(self.L.qsa_oracle_e4m3_to_double(int(code) & 0xFF))
+
+    def decode_fp8(self, q, k8, k_scale: float, page_table, seq_lens, W: int, scale: float = SCALE,
+                   threads: int = 0) -> np.ndarray:
+        """fp64 scores [B, Q, W] over an fp8 E4M3 key cache k8 (uint8 codes
+        [pages, page_size, 1, 128]) with dequantisation scale k_scale."""
+        qb, qs = _bf16_bits(q)
+        if len(qs) != 4 or qs[3] != 1:
+            raise ValueError("q must be [B, Q, 4, 128] with unit feature stride")
+        if hasattr(k8, "cpu"):
+            import torch
+            k8 = k8.detach().cpu()
+            if k8.dtype != torch.uint8:
+                k8 = k8.view(torch.uint8)
+            kst = tuple(k8.stride())
+            kb = k8.numpy()
+        else:
+            kb = np.asarray(k8, dtype=np.uint8)
+            kst = tuple(kb.strides)
+        if len(kst) != 4 or kst[3] != 1:
+            raise ValueError("k8 must be [pages, page_size, 1, 128] with unit feature stride")
+        pt, sl = _i32(page_table), _i32(seq_lens)
+        B, Q = qb.shape[0], qb.shape[1]
+        out = np.empty((B, Q, W), dtype=np.float64)
+        self.L.qsa_oracle_decode_fp8(_ptr(qb), qs[0], qs[1], qs[2], _ptr(kb), float(k_scale), kb.shape[0],
+                                     kb.shape[1], kst[0], kst[1], _ptr(pt), pt.shape[1], pt.shape[1],
+                                     _ptr(sl), B, Q, float(scale), _ptr(out), W, threads)
         return out
 
     def decode_entries(self, q, k_cache, page_table, seq_lens, b, i, n, scale: float = SCALE,

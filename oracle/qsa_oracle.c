@@ -129,14 +129,39 @@ void qsa_oracle_prefill_intervals(const int32_t *cu_seqlens_q, const int32_t *se
 
 /* ------------------------------------------------------------- the score */
 
+/* Value of an fp8 E4M3 code (the e4m3 format with no infinities: 1 sign
+ * bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0 holds the
+ * subnormals m * 2^-9; the codes with all exponent and mantissa bits set are
+ * NaN; the largest finite magnitude is 1.75 * 2^8 = 448). */
+double qsa_oracle_e4m3_to_double(uint8_t code) {
+    int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* A key row as exact doubles: bf16 elements, or fp8 E4M3 elements times the
+ * cache's dequantisation scale k_scale (the cache stores e4m3(bf16(k) /
+ * k_scale): vLLM qsa_prepare.py, "_to_dst_dtype", rounds to bf16 first, then
+ * scales for an fp8 destination). */
+static void key_row_bf16(const uint16_t *k_row, double *k) {
+    for (int e = 0; e < QSA_DIM; ++e) k[e] = bf16_to_double(k_row[e]);
+}
+
+static void key_row_e4m3(const uint8_t *k_row, double k_scale, double *k) {
+    for (int e = 0; e < QSA_DIM; ++e) k[e] = qsa_oracle_e4m3_to_double(k_row[e]) * k_scale;
+}
+
 /* scale * sum_h max(0, q_h . k) for one query row (4 heads) and one key. */
 static double head_sum_score(const uint16_t *q_row, int64_t q_stride_h,
-                             const uint16_t *k_row, double scale) {
+                             const double *k, double scale) {
     double s = 0.0;
     for (int h = 0; h < QSA_HEADS; ++h) {
         const uint16_t *qh = q_row + h * q_stride_h;
         double d = 0.0;
-        for (int c = 0; c < QSA_DIM; ++c) d += bf16_to_double(qh[c]) * bf16_to_double(k_row[c]);
+        for (int c = 0; c < QSA_DIM; ++c) d += bf16_to_double(qh[c]) * k[c];
         s += d > 0.0 ? d : 0.0;
     }
     return scale * s;
@@ -148,6 +173,7 @@ typedef struct {
     const int32_t *page_table; int64_t pt_stride, max_pages;
     const int32_t *seq_lens; int64_t B, Q;
     double scale;
+    const uint8_t *k8; double k_scale;   /* fp8 cache when k8 != NULL (then k_cache is unused) */
 } decode_args;
 
 /* Score of decode row (b, i) against compressed key n, or -inf when masked. */
@@ -159,9 +185,12 @@ static double decode_entry(const decode_args *a, int64_t b, int64_t i, int64_t n
     if (logical_page >= a->max_pages) return -INFINITY;
     int64_t page = a->page_table[b * a->pt_stride + logical_page];
     if (page < 0 || page >= a->num_pages) return -INFINITY;
-    const uint16_t *k_row = a->k_cache + page * a->k_page_stride + (n % a->page_size) * a->k_row_stride;
     const uint16_t *q_row = a->q + b * a->q_sb + i * a->q_st;
-    return head_sum_score(q_row, a->q_sh, k_row, a->scale);
+    int64_t row_off = page * a->k_page_stride + (n % a->page_size) * a->k_row_stride;
+    double k[QSA_DIM];
+    if (a->k8) key_row_e4m3(a->k8 + row_off, a->k_scale, k);
+    else key_row_bf16(a->k_cache + row_off, k);
+    return head_sum_score(q_row, a->q_sh, k, a->scale);
 }
 
 typedef struct { decode_args a; double *out; int64_t W; } decode_full_ctx;
@@ -182,7 +211,23 @@ void qsa_oracle_decode(const uint16_t *q, int64_t q_sb, int64_t q_st, int64_t q_
                        const int32_t *seq_lens, int64_t B, int64_t Q, double scale,
                        double *out, int64_t W, int nthreads) {
     decode_full_ctx c = {{q, q_sb, q_st, q_sh, k_cache, num_pages, page_size, k_page_stride,
-                          k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale},
+                          k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale,
+                          NULL, 0.0},
+                         out, W};
+    parallel_for(B * Q, nthreads, decode_rows, &c);
+}
+
+/* qsa_oracle_decode over an fp8 E4M3 key cache (strides in bytes = elements)
+ * with dequantisation scale k_scale. */
+void qsa_oracle_decode_fp8(const uint16_t *q, int64_t q_sb, int64_t q_st, int64_t q_sh,
+                           const uint8_t *k8, double k_scale, int64_t num_pages, int64_t page_size,
+                           int64_t k_page_stride, int64_t k_row_stride,
+                           const int32_t *page_table, int64_t pt_stride, int64_t max_pages,
+                           const int32_t *seq_lens, int64_t B, int64_t Q, double scale,
+                           double *out, int64_t W, int nthreads) {
+    decode_full_ctx c = {{q, q_sb, q_st, q_sh, NULL, num_pages, page_size, k_page_stride,
+                          k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale,
+                          k8, k_scale},
                          out, W};
     parallel_for(B * Q, nthreads, decode_rows, &c);
 }
@@ -203,7 +248,8 @@ void qsa_oracle_decode_entries(const uint16_t *q, int64_t q_sb, int64_t q_st, in
                                const int64_t *bb, const int64_t *ii, const int64_t *nn,
                                int64_t count, double *out, int nthreads) {
     decode_entries_ctx c = {{q, q_sb, q_st, q_sh, k_cache, num_pages, page_size, k_page_stride,
-                             k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale},
+                             k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale,
+                             NULL, 0.0},
                             bb, ii, nn, out};
     parallel_for(count, nthreads, decode_entries_range, &c);
 }
@@ -221,7 +267,9 @@ static double prefill_entry(const prefill_args *a, int64_t t, int64_t j) {
     int64_t hi = a->ke[t] < a->Nk ? a->ke[t] : a->Nk;
     int64_t n = (int64_t)a->ks[t] + j;
     if (j < 0 || n < lo || n >= hi) return -INFINITY;
-    return head_sum_score(a->q + t * a->q_st, a->q_sh, a->k + n * a->k_stride, a->scale);
+    double k[QSA_DIM];
+    key_row_bf16(a->k + n * a->k_stride, k);
+    return head_sum_score(a->q + t * a->q_st, a->q_sh, k, a->scale);
 }
 
 typedef struct { prefill_args a; double *out; int64_t W; } prefill_full_ctx;

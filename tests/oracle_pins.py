@@ -14,7 +14,12 @@ when the oracle disagrees with:
   visibility comes from the writer simulation, sums are Python integers);
 * closed forms, invariants and cross-entry identities of the definition in
   the QSA docs (MATE, section "MQA score");
-* a full sort for the top-k selection.
+* a full sort for the top-k selection;
+* for the fp8 E4M3 key cache (vLLM qsa_cache.py, the state backend's fp8
+  cache dtypes; vLLM qsa_prepare.py, "_to_dst_dtype"): torch's own E4M3
+  decoding of all 256 codes and the format's fixed values, exact integer
+  brute force with keys that E4M3 holds exactly, and the bf16 entry on keys
+  dequantised by torch.
 
 The same functions run against deliberately broken builds of the oracle
 (``test_oracle_mutants.py``) to show that each plausible mistake trips a pin.
@@ -355,6 +360,71 @@ def pin_topk_ties_and_padding(orc):
     assert orc.topk(s2, np.array([4], dtype=np.int32), 3)[0].tolist() == [1, 3, -1]
 
 
+# ---------------------------------------------------------------- fp8 cache
+
+def pin_e4m3_decoder(orc):
+    """Every E4M3 code against torch's float8_e4m3fn decoding, and the
+    format's fixed points (no infinities, NaN at 0x7f / 0xff, largest finite
+    value 448, smallest subnormal 2^-9, smallest normal 2^-6, 1.0 = 0x38)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([orc.e4m3_to_double(c) for c in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF])
+    assert got[0x7E] == 448.0 and got[0xFE] == -448.0
+    assert got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6 and got[0x38] == 1.0
+    assert got[0x00] == 0.0 and math.copysign(1.0, got[0x80]) == -1.0
+
+
+def _e4m3_codes(x: torch.Tensor) -> torch.Tensor:
+    return x.to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def pin_fp8_decode_exact_bruteforce(orc):
+    """Integer keys (exact in E4M3) with k_scale 3 and 1/2: the score is
+    k_scale times the exact integer brute force."""
+    rng = np.random.default_rng(11)
+    cases = [(1, 1, 8, [37]), (3, 4, 8, [70, 41, 2]), (2, 3, 16, [130, 75])]
+    for B, Q, ps, lens in cases:
+        q, kc, table, sl, W = paged_case(rng, B, Q, ps, lens)
+        k8 = _e4m3_codes(kc)
+        want = brute_decode(q, kc, table.numpy(), sl.numpy(), W)
+        for ks in (3.0, 0.5):
+            got = orc.decode_fp8(q, k8, ks, table, sl, W, scale=1.0, threads=2)
+            assert np.array_equal(got, want * ks), (B, Q, ps, lens, ks)
+
+
+def pin_fp8_matches_bf16_on_dequantised_keys(orc):
+    """Random finite codes (subnormals and both zeros included) with a
+    power-of-two k_scale: every dequantised key is exact in bf16, so the fp8
+    entry must equal the bf16 entry on the keys torch dequantises."""
+    g = torch.Generator().manual_seed(12)
+    B, Q, ps, lens = 3, 2, 16, [300, 41, 200]
+    pages = sum(-(-L // (4 * ps)) for L in lens) + 1
+    codes = torch.randint(0, 256, (pages, ps, 1, 128), generator=g, dtype=torch.int32)
+    codes[(codes == 0x7F) | (codes == 0xFF)] = 0x00
+    codes[0, 0, 0, :8] = torch.tensor([0x00, 0x80, 0x01, 0x81, 0x07, 0x08, 0x7E, 0xFE])
+    k8 = codes.to(torch.uint8)
+    ks = 2.0 ** -5
+    kbf = (k8.view(torch.float8_e4m3fn).to(torch.float32) * ks).to(torch.bfloat16)
+    assert torch.equal(kbf.to(torch.float64), k8.view(torch.float8_e4m3fn).to(torch.float64) * ks)
+    q = torch.randn(B, Q, 4, 128, generator=g).to(torch.bfloat16)
+    table = torch.full((B, max(-(-L // (4 * ps)) for L in lens)), -1, dtype=torch.int32)
+    at = 0
+    for b, L in enumerate(lens):
+        n = -(-L // (4 * ps))
+        table[b, :n] = torch.arange(at, at + n, dtype=torch.int32)
+        at += n
+    sl = torch.tensor(lens, dtype=torch.int32)
+    W = max(lens) // 4 + 5
+    got = orc.decode_fp8(q, k8, ks, table, sl, W, threads=2)
+    want = orc.decode(q, kbf, table, sl, W, threads=2)
+    assert np.array_equal(np.isneginf(got), np.isneginf(want))
+    assert np.array_equal(got, want)
+    assert np.isfinite(got).sum() > 0
+
+
 ALL_PINS = [
     pin_visible_blocks_follow_cache_writer,
     pin_decode_positions_are_last_tokens,
@@ -367,4 +437,7 @@ ALL_PINS = [
     pin_cross_entry_identities,
     pin_topk_against_full_sort,
     pin_topk_ties_and_padding,
+    pin_e4m3_decoder,
+    pin_fp8_decode_exact_bruteforce,
+    pin_fp8_matches_bf16_on_dequantised_keys,
 ]

@@ -31,6 +31,13 @@ MUTANTS = {
     "top-k ties to the higher column": ("return (a->j > b->j) - (a->j < b->j);",
                                         "return (a->j < b->j) - (a->j > b->j);"),
     "top-k selects masked blocks": ("if (!(v > -INFINITY)) continue;", "if (v != v) continue;"),
+    "fp8 dequantisation scale dropped": ("k[e] = qsa_oracle_e4m3_to_double(k_row[e]) * k_scale;",
+                                         "k[e] = qsa_oracle_e4m3_to_double(k_row[e]);"),
+    "e4m3 exponent bias off by one": ("else v = ldexp(1.0 + m / 8.0, e - 7);",
+                                      "else v = ldexp(1.0 + m / 8.0, e - 8);"),
+    "e4m3 subnormals read as normals": ("if (e == 0) v = ldexp((double)m, -9);",
+                                        "if (e == 0) v = ldexp(1.0 + m / 8.0, -7);"),
+    "e4m3 sign ignored": ("return sign ? -v : v;", "return v;"),
     "top-k keeps the smallest": ("if (a->v > b->v) return -1;\n    if (a->v < b->v) return 1;",
                                  "if (a->v < b->v) return -1;\n    if (a->v > b->v) return 1;"),
 }

@@ -48,11 +48,12 @@ PUBLISHED = {  # the vLLM PR's GB300 numbers for the same workload shapes (conte
 
 # ------------------------------------------------------------------ accounting
 
-def decode_bytes(seq_lens, dql: int) -> int:
-    """Algorithmic bytes of one decode step: the visible bf16 keys, the fp32
-    scores of the visible blocks and the bf16 queries."""
+def decode_bytes(seq_lens, dql: int, key_bytes: int = 256) -> int:
+    """Algorithmic bytes of one decode step: the visible keys (256 bytes each
+    in bf16, 128 in fp8), the fp32 scores of the visible blocks and the bf16
+    queries."""
     keys = sum(int(L) // 4 for L in seq_lens)
-    return keys * 256 + dql * keys * 4 + len(seq_lens) * dql * 1024
+    return keys * key_bytes + dql * keys * 4 + len(seq_lens) * dql * 1024
 
 
 def prefill_flops(ks, ke) -> int:
@@ -153,14 +154,19 @@ class DecodeBench:
     kernel = "decode_kernel"
     bound = "hbm"
 
-    def __init__(self, cfg: int, dev: torch.device, seed: int):
+    def __init__(self, cfg: int, dev: torch.device, seed: int, fp8: bool = False):
         import sparse_attention_block_qsa_b200 as qsa
         self.qsa = qsa
         self.inp = wl.make_config(cfg, seed=seed)
         d = self.inp
-        self.name = d.name
-        self.units = decode_bytes(d.seq_lens.tolist(), d.Q)        # algorithmic bytes per step
-        per_copy = (d.q.numel() + d.k_cache.numel()) * 2 + d.B * d.Q * d.W * 4
+        self.fp8 = fp8
+        self.k_scale = 1.0
+        if fp8:   # the same keys in the fp8 E4M3 cache format
+            d.k_cache, self.k_scale = wl.e4m3_cache(d.k_cache)
+        kb = d.k_cache.element_size()
+        self.name = d.name + ("_fp8" if fp8 else "")
+        self.units = decode_bytes(d.seq_lens.tolist(), d.Q, 128 * kb)   # algorithmic bytes per step
+        per_copy = d.q.numel() * 2 + d.k_cache.numel() * kb + d.B * d.Q * d.W * 4
         self.copies = max(2, math.ceil(2 * L2_BYTES / per_copy))
         self.dev = dev
         self.bufs = []
@@ -168,16 +174,22 @@ class DecodeBench:
             self.bufs.append((d.q.to(dev), d.k_cache.to(dev), d.page_table.to(dev), d.seq_lens.to(dev),
                               torch.empty((d.B, d.Q, d.W), dtype=torch.float32, device=dev)))
         self.launches_per_step = 1
-        self.h2d = (d.q.numel() + d.k_cache.numel()) * 2 + (d.page_table.numel() + d.seq_lens.numel()) * 4
+        self.h2d = d.q.numel() * 2 + d.k_cache.numel() * kb + (d.page_table.numel() + d.seq_lens.numel()) * 4
         self.d2h = d.B * d.Q * d.W * 4
-        self.config = {"workload": d.name, "requests": d.B, "query_tokens": d.Q, "page_size": d.page_size,
+        self.dtype = "fp8e4m3 keys, bf16 queries" if fp8 else "bf16"
+        self.config = {"workload": self.name, "kv_cache_dtype": "fp8_e4m3" if fp8 else "bf16", "requests": d.B, "query_tokens": d.Q, "page_size": d.page_size,
                        "context_tokens": d.meta["context_tokens"], "W": d.W, "input_copies": self.copies,
                        "l2": f"steps rotate over {self.copies} input copies "
                              f"({self.copies * per_copy / 2**20:.0f} MiB > 2x L2)"}
 
+    def _launch(self, q, kc, pt, sl, out):
+        if self.fp8:
+            self.qsa.mqa_decode_fp8(q, kc, self.k_scale, pt, sl, self.inp.W, out=out)
+        else:
+            self.qsa.mqa_decode(q, kc, pt, sl, self.inp.W, out=out)
+
     def step(self, i: int):
-        q, kc, pt, sl, out = self.bufs[i % self.copies]
-        self.qsa.mqa_decode(q, kc, pt, sl, self.inp.W, out=out)
+        self._launch(*self.bufs[i % self.copies])
 
     def throughput(self, seconds_per_step: float) -> float:
         return self.units / seconds_per_step / 1e9   # GB/s
@@ -193,13 +205,16 @@ class DecodeBench:
         q, kc, pt, sl, out = self.bufs[i % self.copies]
         for dst, src in zip((q, kc, pt, sl), self.host):
             dst.copy_(src, non_blocking=True)
-        self.qsa.mqa_decode(q, kc, pt, sl, self.inp.W, out=out)
+        self._launch(q, kc, pt, sl, out)
         self.host_out.copy_(out, non_blocking=True)
 
     def oracle_step(self, threads: int = 0):
         import oracle
         d = self.inp
-        oracle.decode(d.q, d.k_cache, d.page_table, d.seq_lens, d.W, threads=threads)
+        if self.fp8:
+            oracle.decode_fp8(d.q, d.k_cache, self.k_scale, d.page_table, d.seq_lens, d.W, threads=threads)
+        else:
+            oracle.decode(d.q, d.k_cache, d.page_table, d.seq_lens, d.W, threads=threads)
 
     def oracle_sample(self):
         return 1.0, "one full step (every score of the batch)"
@@ -278,8 +293,10 @@ class PrefillBench:
             oracle.topk(s, np.full(s.shape[0], p.W, dtype=np.int32), wl.TOPK_K, threads=threads)
 
 
-def make_bench(cfg: int, dev, seed: int):
-    return DecodeBench(cfg, dev, seed) if cfg in (1, 2, 3) else PrefillBench(cfg, dev, seed)
+def make_bench(cfg: int, dev, seed: int, fp8: bool = False):
+    if fp8 and cfg not in (1, 2, 3):
+        raise ValueError("the fp8 key cache applies to the decode configurations 1-3")
+    return DecodeBench(cfg, dev, seed, fp8) if cfg in (1, 2, 3) else PrefillBench(cfg, dev, seed)
 
 
 # ------------------------------------------------------------------ timing
@@ -395,7 +412,7 @@ def run_reference(args, rank: int, world: int):
         return
     dev = torch.device("cpu")
     import oracle
-    inp_bench = _HostOnly(args.config)
+    inp_bench = _HostOnly(args.config, args.kv_fp8)
     threads = oracle.default_threads()
     frac, what = inp_bench.oracle_sample()
     for _ in range(args.warmup):
@@ -419,15 +436,20 @@ def run_reference(args, rank: int, world: int):
 class _HostOnly:
     """Inputs and accounting of a workload without any GPU state."""
 
-    def __init__(self, cfg: int):
+    def __init__(self, cfg: int, fp8: bool = False):
         self.cfg = cfg
         self.inp = wl.make_config(cfg)
+        self.fp8 = fp8 and cfg in (1, 2, 3)
+        self.k_scale = 1.0
         if cfg in (1, 2, 3):
             d = self.inp
-            self.units = decode_bytes(d.seq_lens.tolist(), d.Q)
+            if self.fp8:
+                d.k_cache, self.k_scale = wl.e4m3_cache(d.k_cache)
+            self.units = decode_bytes(d.seq_lens.tolist(), d.Q, 128 * d.k_cache.element_size())
             self.unit = "GB/s"
-            self.config = {"workload": d.name, "requests": d.B, "query_tokens": d.Q, "page_size": d.page_size,
-                           "W": d.W}
+            self.config = {"workload": d.name + ("_fp8" if self.fp8 else ""),
+                           "kv_cache_dtype": "fp8_e4m3" if self.fp8 else "bf16", "requests": d.B,
+                           "query_tokens": d.Q, "page_size": d.page_size, "W": d.W}
         else:
             import oracle
             p = self.inp
@@ -459,6 +481,7 @@ def main():
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-fp8", action="store_true", help="decode over the fp8 E4M3 key cache")
     ap.add_argument("--soak", type=float, default=1.5, help="seconds of load before the timed region")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -477,7 +500,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
 
-    b = make_bench(args.config, dev, seed=rank)
+    b = make_bench(args.config, dev, seed=rank, fp8=args.kv_fp8)
     for i in range(args.warmup):
         b.step(i)
     torch.cuda.synchronize()
@@ -507,7 +530,7 @@ def main():
                     "traffic": read_traffic(b.kernel, b.name), "kernel": b.kernel,
                     "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst figure)"
                     if peaks["source"] == "measured" else "fallback"}
-        pub = PUBLISHED.get(args.config)
+        pub = None if args.kv_fp8 else PUBLISHED.get(args.config)
         cfg = dict(b.config)
         if pub:
             cfg["published_reference"] = pub[2]
@@ -515,7 +538,7 @@ def main():
                 "warmup": args.warmup, "ms_per_step": per_step * 1e3, "us_per_step": per_step * 1e6,
                 "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": (value / pub[1]) if pub and pub[0] == b.unit else None,
-                "dtype": "bf16", "data": "synthetic", "config": cfg,
+                "dtype": getattr(b, "dtype", "bf16"), "data": "synthetic", "config": cfg,
                 "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                 "roofline": roofline,
                 "e2e": {"value": b.throughput(e2e_s) * world, "unit": b.unit, "h2d_bytes_per_step": b.h2d,

@@ -119,6 +119,30 @@ qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_
                             float* out, int64_t out_stride_b, int64_t out_stride_t, int32_t W, void* stream);
 
 /*
+ * qsa_mqa_decode_fp8 - qsa_mqa_decode over an fp8 E4M3 compressed key cache.
+ *
+ * The cache dtype is the optional e4m3 indexer cache of vLLM qsa_cache.py
+ * (the QSA state backend's cache dtypes "fp8" / "fp8_e4m3"); its writer
+ * (vLLM qsa_prepare.py, "_to_dst_dtype") rounds a key to bf16, divides it by
+ * the cache scale and stores the E4M3 code.  Key element c of a row is read
+ * as E4M3(code) * k_scale, and the score is the bf16 one on those keys:
+ * scale * sum_h max(0, q_h . k).  Arguments as qsa_mqa_decode, except:
+ *
+ *   k_cache    E4M3 codes (one byte each) [num_pages, page_size, 1, 128],
+ *              strides in bytes: 16-byte aligned, k_row_stride and
+ *              k_page_stride multiples of 16, k_row_stride >= 128.  The NaN
+ *              codes 0x7f / 0xff are outside the contract (the writer does
+ *              not produce them for finite keys).
+ *   k_scale    dequantisation scale: finite and > 0 (scale * k_scale finite).
+ */
+qsa_status_t qsa_mqa_decode_fp8(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
+                                const void* k_cache, float k_scale, int64_t num_pages, int32_t page_size,
+                                int64_t k_page_stride, int64_t k_row_stride, const int32_t* page_table,
+                                int64_t pt_stride, int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t Q,
+                                float scale, float* out, int64_t out_stride_b, int64_t out_stride_t, int32_t W,
+                                void* stream);
+
+/*
  * qsa_mqa_prefill - prefill scores of packed query rows against shared keys
  * with one key interval per row.
  *

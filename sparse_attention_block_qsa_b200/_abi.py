@@ -26,6 +26,8 @@ SIGNATURES = {
     "qsa_selftest_bounded_wait": (C.c_int, [C.c_uint64, _i32, _vp]),
     "qsa_mqa_decode": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _i64, _i32, _i64, _i64, _vp, _i64, _i32,
                                  _vp, _i32, _i32, _f32, _vp, _i64, _i64, _i32, _vp]),
+    "qsa_mqa_decode_fp8": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _f32, _i64, _i32, _i64, _i64, _vp, _i64,
+                                     _i32, _vp, _i32, _i32, _f32, _vp, _i64, _i64, _i32, _vp]),
     "qsa_mqa_prefill": (C.c_int, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f32, _vp, _i64,
                                   _i32, _vp]),
     "qsa_prefill_intervals": (C.c_int, [_vp, _vp, _vp, _i32, _i64, _vp, _vp, _vp]),
@@ -103,13 +105,8 @@ def selftest_bounded_wait(timeout_ns: int, arrive: bool, stream=None) -> None:
                                                                        _stream(stream)))
 
 
-def mqa_decode(q: torch.Tensor, k_cache: torch.Tensor, page_table: torch.Tensor, seq_lens: torch.Tensor,
-               W: int, scale: float = SCALE, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Decode / spec-decode scores: q bf16 [B, Q, 4, 128], k_cache bf16
-    [pages, page_size, 1, 128], page_table int32 [B, max_pages], seq_lens int32
-    [B] (tokens) -> out fp32 [B, Q, W]."""
+def _decode_checks(q, k_cache, page_table, seq_lens, W, out):
     _need(q, "q", torch.bfloat16, 4)
-    _need(k_cache, "k_cache", torch.bfloat16, 4)
     _need(page_table, "page_table", torch.int32, 2)
     _need(seq_lens, "seq_lens", torch.int32, 1)
     B, Q = q.shape[0], q.shape[1]
@@ -124,9 +121,37 @@ def mqa_decode(q: torch.Tensor, k_cache: torch.Tensor, page_table: torch.Tensor,
         raise ValueError("page_table, seq_lens and out need a unit innermost stride")
     if out.shape[:2] != (B, Q) or page_table.shape[0] != B or seq_lens.shape[0] != B:
         raise ValueError("batch shapes of q, page_table, seq_lens and out disagree")
+    return B, Q, out
+
+
+def mqa_decode(q: torch.Tensor, k_cache: torch.Tensor, page_table: torch.Tensor, seq_lens: torch.Tensor,
+               W: int, scale: float = SCALE, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode / spec-decode scores: q bf16 [B, Q, 4, 128], k_cache bf16
+    [pages, page_size, 1, 128], page_table int32 [B, max_pages], seq_lens int32
+    [B] (tokens) -> out fp32 [B, Q, W]."""
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    B, Q, out = _decode_checks(q, k_cache, page_table, seq_lens, W, out)
     _check("qsa_mqa_decode", lib().qsa_mqa_decode(
         _ptr(q), q.stride(0), q.stride(1), q.stride(2),
         _ptr(k_cache), k_cache.shape[0], k_cache.shape[1], k_cache.stride(0), k_cache.stride(1),
+        _ptr(page_table), page_table.stride(0), page_table.shape[1], _ptr(seq_lens), B, Q, scale,
+        _ptr(out), out.stride(0), out.stride(1), out.shape[2], _stream(stream)))
+    return out
+
+
+def mqa_decode_fp8(q: torch.Tensor, k_cache: torch.Tensor, k_scale: float, page_table: torch.Tensor,
+                   seq_lens: torch.Tensor, W: int, scale: float = SCALE, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """mqa_decode over an fp8 E4M3 key cache: k_cache float8_e4m3fn (or uint8
+    codes) [pages, page_size, 1, 128] holding e4m3(bf16(k) / k_scale); keys
+    are read as E4M3 value * k_scale (k_scale > 0)."""
+    if isinstance(k_cache, torch.Tensor) and k_cache.dtype == torch.float8_e4m3fn:
+        k_cache = k_cache.view(torch.uint8)
+    _need(k_cache, "k_cache", torch.uint8, 4)
+    B, Q, out = _decode_checks(q, k_cache, page_table, seq_lens, W, out)
+    _check("qsa_mqa_decode_fp8", lib().qsa_mqa_decode_fp8(
+        _ptr(q), q.stride(0), q.stride(1), q.stride(2),
+        _ptr(k_cache), float(k_scale), k_cache.shape[0], k_cache.shape[1], k_cache.stride(0), k_cache.stride(1),
         _ptr(page_table), page_table.stride(0), page_table.shape[1], _ptr(seq_lens), B, Q, scale,
         _ptr(out), out.stride(0), out.stride(1), out.shape[2], _stream(stream)))
     return out

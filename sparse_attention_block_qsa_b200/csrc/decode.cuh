@@ -32,7 +32,20 @@
 // Tensor-core throughput is not the limit here (at most 4 of the 16 rows
 // carry data for one token); the warp-level MMA is used because its operands
 // come from registers, which lets the key loads bypass shared memory.
+//
+// fp8 E4M3 cache (vLLM qsa_cache.py, the state backend's fp8 cache dtypes;
+// vLLM qsa_prepare.py, "_to_dst_dtype": stored = e4m3(bf16(k) / k_scale)):
+// a lane reads 8 bytes per chunk instead of 16, with twice the tiles in
+// flight (the same 256 bytes per lane).  Every E4M3 value is exact in fp16,
+// so keys are widened with one conversion per pair and the MMA runs on fp16.
+// The query rows are made fp16 exactly: each row is multiplied by the power
+// of two that puts its largest magnitude in [2^15, 2^16) (exact for every
+// element within 29 binades of it), and the row's accumulators are multiplied
+// back before the ReLU sum.  k_scale > 0 is folded into the score multiplier.
 #pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "sm100.cuh"
 
@@ -40,7 +53,7 @@ namespace qsa {
 namespace decode {
 
 constexpr int TILE = 8;                 // keys per tile (mma.sync N)
-constexpr int BATCH = 4;                // tiles in flight per warp
+constexpr int BATCH = 4;                // tiles in flight per warp (bf16 keys; fp8 keys: 2 * BATCH)
 constexpr int WARPS = 16;
 constexpr int NUM_THREADS = WARPS * 32;
 constexpr int MAX_B = 8192;             // requests per launch (prefix in shared memory)
@@ -48,8 +61,9 @@ constexpr int MAX_B = 8192;             // requests per launch (prefix in shared
 struct Params {
   const uint16_t* q;        // bf16 bits
   int64_t q_sb, q_st, q_sh;
-  const uint16_t* k_cache;  // bf16 bits
-  int64_t k_page_stride, k_row_stride;
+  const uint16_t* k_cache;  // bf16 bits (bf16 cache)
+  const uint8_t* k8;        // E4M3 codes (fp8 cache)
+  int64_t k_page_stride, k_row_stride;  // in elements
   int64_t num_pages;
   const int32_t* page_table;
   int64_t pt_stride;
@@ -58,7 +72,7 @@ struct Params {
   int32_t B;
   int32_t Q;
   int32_t log2_ps;
-  float scale;
+  float scale;              // fp8 cache: scale * k_scale
   float* out;
   int64_t out_sb;
   int64_t out_st;
@@ -88,6 +102,42 @@ __device__ __forceinline__ uint4 ld_stream16(const void* ptr) {
   return v;
 }
 
+__device__ __forceinline__ uint2 ld_stream8(const void* ptr) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(ptr));
+  return v;
+}
+
+__device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two E4M3 codes (low byte = lower feature) -> fp16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// bf16x2 word -> fp16x2 word of the two values times dn (a power of two).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float dn) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(w << 16) * dn, __uint_as_float(w & 0xffff0000u) * dn);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Power-of-two factors for a query row whose largest bf16 magnitude (bits
+// without the sign) is m: dn = 2^(142 - E) with E its exponent field, so the
+// row times dn has its largest magnitude in [2^15, 2^16), and up = 1 / dn.
+// E is held at >= 16 so that both factors are normal floats.
+__device__ __forceinline__ void row_factors(uint32_t m, float& dn, float& up) {
+  const int e = max((int)(m >> 7), 16);
+  dn = __uint_as_float((uint32_t)(269 - e) << 23);
+  up = __uint_as_float((uint32_t)(e - 15) << 23);
+}
+
 __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
@@ -105,7 +155,11 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint
 // eight k-steps and four lanes every feature is used exactly once.
 
 // Query fragments of request b: A = 16 rows (row = head * 4 + token) x 128.
-__device__ __forceinline__ void load_queries(const Params& p, int b, int lane, uint32_t (&a)[8][4]) {
+// fp8 cache: fp16 fragments of the scaled rows, and in up0 / up1 the factors
+// that undo the scaling of rows g and g + 8.
+template <bool FP8>
+__device__ __forceinline__ void load_queries(const Params& p, int b, int lane, uint32_t (&a)[8][4], float& up0,
+                                             float& up1) {
   const int g = lane >> 2, c = lane & 3;
   const int t = g & 3, h = g >> 2;  // rows g and g + 8: heads h and h + 2 of token t
   // Rows of tokens t >= Q read token Q - 1 instead (no branch, so the loads
@@ -120,6 +174,27 @@ __device__ __forceinline__ void load_queries(const Params& p, int b, int lane, u
     w0[4 * i] = x.x; w0[4 * i + 1] = x.y; w0[4 * i + 2] = x.z; w0[4 * i + 3] = x.w;
     w1[4 * i] = y.x; w1[4 * i + 1] = y.y; w1[4 * i + 2] = y.z; w1[4 * i + 3] = y.w;
   }
+  if constexpr (FP8) {
+    uint32_t m0 = 0, m1 = 0;  // largest magnitude bits of rows g and g + 8 (this lane's 32 features)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      m0 = max(m0, max(w0[i] & 0x7fffu, (w0[i] >> 16) & 0x7fffu));
+      m1 = max(m1, max(w1[i] & 0x7fffu, (w1[i] >> 16) & 0x7fffu));
+    }
+    // the row's four lanes c = 0..3 differ in the low two lane bits
+    m0 = max(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+    m1 = max(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+    m0 = max(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+    m1 = max(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
+    float dn0, dn1;
+    row_factors(m0, dn0, up0);
+    row_factors(m1, dn1, up1);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      w0[i] = bf16x2_to_f16x2(w0[i], dn0);
+      w1[i] = bf16x2_to_f16x2(w1[i], dn1);
+    }
+  }
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     a[s][0] = w0[2 * s];      // row g,     k = 2c + {0,1}
@@ -129,7 +204,9 @@ __device__ __forceinline__ void load_queries(const Params& p, int b, int lane, u
   }
 }
 
+template <bool FP8>
 __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) {
+  constexpr int NB = FP8 ? 2 * BATCH : BATCH;  // tiles in flight per warp
   extern __shared__ int32_t prefix[];  // prefix[b]: tiles before request b
   __shared__ uint32_t red[WARPS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -289,7 +366,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   const int key = 2 * c + (lane >> 4);  // key of a tile this lane stores
   const int ps_mask = (1 << p.log2_ps) - 1;
   uint32_t qa[8][4];
-  load_queries(p, b, lane, qa);
+  float up0 = 1.f, up1 = 1.f;
+  load_queries<FP8>(p, b, lane, qa, up0, up1);
   int L = __ldg(p.seq_lens + b);
   int nt_b = (int)(pfx(b + 1) - pfx(b));
   // Page of tile j0 + lane of the current request, read 32 tiles ahead so
@@ -306,24 +384,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   fetch_entries();
 
   while (left > 0) {
-    const int cnt = (int)min((uint32_t)min(min(BATCH, nt_b - j), 32 - (j - j0)), left);
-    uint4 kv[BATCH][4];
-    int ent[BATCH];
+    const int cnt = (int)min((uint32_t)min(min(NB, nt_b - j), 32 - (j - j0)), left);
+    uint4 kv[FP8 ? 1 : NB][4];   // bf16: chunk i = 16 bytes
+    uint2 kv8[FP8 ? NB : 1][4];  // fp8: chunk i = 8 bytes
+    uint32_t valid = 0;  // bit u: tile u has a page
 #pragma unroll
-    for (int u = 0; u < BATCH; ++u) {
-      ent[u] = __shfl_sync(0xffffffffu, entry, (j - j0 + u) & 31);
+    for (int u = 0; u < NB; ++u) {
+      const int ent = __shfl_sync(0xffffffffu, entry, (j - j0 + u) & 31);
       // tiles past the request's pages (logical page >= max_pages) and
       // entries outside the pool are invalid
       const bool in_table = (((j + u) * TILE) >> p.log2_ps) < p.max_pages;
-      if (!(in_table && ent[u] >= 0 && (int64_t)ent[u] < p.num_pages)) ent[u] = -1;
-      if (u < cnt && ent[u] >= 0) {
-        const int row = ((j + u) * TILE + g) & ps_mask;
-        const uint16_t* kr = p.k_cache + (int64_t)ent[u] * p.k_page_stride + (int64_t)row * p.k_row_stride;
+      const bool ok = in_table && ent >= 0 && (int64_t)ent < p.num_pages;
+      valid |= ok ? 1u << u : 0u;
+      const int row = ((j + u) * TILE + g) & ps_mask;
+      const int64_t off = (int64_t)ent * p.k_page_stride + (int64_t)row * p.k_row_stride;
+      if constexpr (FP8) {
+        if (u < cnt && ok) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) kv[u][i] = ld_stream16(kr + 8 * (c + 4 * i));
+          for (int i = 0; i < 4; ++i) kv8[u][i] = ld_stream8(p.k8 + off + 8 * (c + 4 * i));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) kv8[u][i] = make_uint2(0, 0);
+        }
       } else {
+        if (u < cnt && ok) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) kv[u][i] = make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 4; ++i) kv[u][i] = ld_stream16(p.k_cache + off + 8 * (c + 4 * i));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) kv[u][i] = make_uint4(0, 0, 0, 0);
+        }
       }
     }
     const int vis = t < p.Q ? visible_of(L, p.Q, t) : 0;
@@ -345,38 +435,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
         fetch_entries();
       }
     }
-    // the batch's MMA chains interleaved by k-step: four independent
+    // the MMA chains of four tiles interleaved by k-step: four independent
     // accumulators keep the tensor pipe busy instead of waiting on one chain
-    float d[BATCH][4];
 #pragma unroll
-    for (int u = 0; u < BATCH; ++u) d[u][0] = d[u][1] = d[u][2] = d[u][3] = 0.f;
+    for (int u0 = 0; u0 < NB; u0 += BATCH) {
+      float d[BATCH][4];
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
+      for (int v = 0; v < BATCH; ++v) d[v][0] = d[v][1] = d[v][2] = d[v][3] = 0.f;
 #pragma unroll
-      for (int u = 0; u < BATCH; ++u) {
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[u]);
-        mma_bf16_16816(d[u], qa[s], w[2 * s], w[2 * s + 1]);
+      for (int s = 0; s < 8; ++s) {
+#pragma unroll
+        for (int v = 0; v < BATCH; ++v) {
+          if constexpr (FP8) {
+            // words 2s, 2s + 1 = bytes 0-3 (s even) or 4-7 (s odd) of chunk s / 2
+            const uint32_t four = (s & 1) ? kv8[u0 + v][s >> 1].y : kv8[u0 + v][s >> 1].x;
+            mma_f16_16816(d[v], qa[s], e4m3x2_to_f16x2(four), e4m3x2_to_f16x2(four >> 16));
+          } else {
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[u0 + v]);
+            mma_bf16_16816(d[v], qa[s], w[2 * s], w[2 * s + 1]);
+          }
+        }
       }
-    }
 #pragma unroll
-    for (int u = 0; u < BATCH; ++u) {
-      if (u < cnt) {
-        // d0/d1: head h, keys 2c and 2c+1; d2/d3: head h + 2
-        float s0 = fmaxf(d[u][0], 0.f) + fmaxf(d[u][2], 0.f);
-        float s1 = fmaxf(d[u][1], 0.f) + fmaxf(d[u][3], 0.f);
-        s0 += __shfl_xor_sync(0xffffffffu, s0, 16);  // the other two heads
-        s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-        const int n = (jb + u) * TILE + key;
-        if (t < p.Q && n < p.W) {
-          const float sc = p.scale * ((lane >> 4) ? s1 : s0);
-          p.out[(int64_t)ob * p.out_sb + (int64_t)t * p.out_st + n] = (ent[u] >= 0 && n < vis) ? sc : -INFINITY;
+      for (int v = 0; v < BATCH; ++v) {
+        const int u = u0 + v;
+        if (u < cnt) {
+          // d0/d1: head h, keys 2c and 2c+1; d2/d3: head h + 2
+          float s0, s1;
+          if constexpr (FP8) {
+            s0 = fmaxf(d[v][0], 0.f) * up0 + fmaxf(d[v][2], 0.f) * up1;
+            s1 = fmaxf(d[v][1], 0.f) * up0 + fmaxf(d[v][3], 0.f) * up1;
+          } else {
+            s0 = fmaxf(d[v][0], 0.f) + fmaxf(d[v][2], 0.f);
+            s1 = fmaxf(d[v][1], 0.f) + fmaxf(d[v][3], 0.f);
+          }
+          s0 += __shfl_xor_sync(0xffffffffu, s0, 16);  // the other two heads
+          s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+          const int n = (jb + u) * TILE + key;
+          if (t < p.Q && n < p.W) {
+            const float sc = p.scale * ((lane >> 4) ? s1 : s0);
+            p.out[(int64_t)ob * p.out_sb + (int64_t)t * p.out_st + n] = ((valid >> u) & 1u) && n < vis ? sc : -INFINITY;
+          }
         }
       }
     }
     if (ob != b) {
       ob = b;
       L = __ldg(p.seq_lens + b);
-      load_queries(p, b, lane, qa);
+      load_queries<FP8>(p, b, lane, qa, up0, up1);
     }
   }
   fill_tail();

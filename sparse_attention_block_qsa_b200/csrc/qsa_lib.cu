@@ -126,7 +126,8 @@ qsa_status_t device_info(int* sms) {
       const void* fn;
       size_t bytes;
     } kernels[] = {
-        {reinterpret_cast<const void*>(qsa::decode::decode_kernel), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<false>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<true>), qsa::decode::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel), qsa::prefill::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_rows_kernel), qsa::topk::ROWS_SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_stream_kernel), qsa::topk::STREAM_SMEM_BYTES},
@@ -373,16 +374,21 @@ qsa_status_t qsa_selftest_bounded_wait(uint64_t timeout_ns, int32_t arrive, void
   return launch_status("self-test kernel");
 }
 
-qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
-                            const void* k_cache, int64_t num_pages, int32_t page_size, int64_t k_page_stride,
-                            int64_t k_row_stride, const int32_t* page_table, int64_t pt_stride, int32_t max_pages,
-                            const int32_t* seq_lens, int32_t B, int32_t Q, float scale, float* out,
-                            int64_t out_stride_b, int64_t out_stride_t, int32_t W, void* stream) {
+// Both cache formats: fp8 selects E4M3 keys (1 byte per element, strides
+// multiples of 16) scaled by k_scale; otherwise bf16 keys and k_scale == 1.
+static qsa_status_t decode_common(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
+                                  const void* k_cache, bool fp8, float k_scale, int64_t num_pages, int32_t page_size,
+                                  int64_t k_page_stride, int64_t k_row_stride, const int32_t* page_table,
+                                  int64_t pt_stride, int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t Q,
+                                  float scale, float* out, int64_t out_stride_b, int64_t out_stride_t, int32_t W,
+                                  void* stream) {
   if (B < 0 || W < 0) return fail(QSA_ERR_INVALID_ARG, "B and W must be non-negative");
   if (Q < 1 || Q > 4) return fail(QSA_ERR_UNSUPPORTED, "Q = %d query tokens per request; 1..4 supported", Q);
   if (page_size != 8 && page_size != 16 && page_size != 32 && page_size != 64)
     return fail(QSA_ERR_UNSUPPORTED, "page_size = %d; supported page sizes are 8, 16, 32 and 64", page_size);
   if (!std::isfinite(scale)) return fail(QSA_ERR_INVALID_ARG, "scale must be finite");
+  if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(scale * k_scale)))
+    return fail(QSA_ERR_INVALID_ARG, "k_scale must be finite and positive, and scale * k_scale finite");
   if (max_pages < 0) return fail(QSA_ERR_INVALID_ARG, "max_pages must be non-negative");
   if (num_pages < 1 || num_pages > INT32_MAX)
     return fail(QSA_ERR_INVALID_ARG, "num_pages = %lld must be in [1, 2^31 - 1]", (long long)num_pages);
@@ -397,10 +403,14 @@ qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_
   for (int i = 0; i < 3; ++i)
     if (qs[i] < 0 || qs[i] % 8 != 0)
       return fail(QSA_ERR_ALIGNMENT, "q strides must be non-negative multiples of 8 (got %lld)", (long long)qs[i]);
-  if (k_row_stride < 128 || k_row_stride % 8 != 0)
-    return fail(QSA_ERR_ALIGNMENT, "k_row_stride = %lld must be a multiple of 8 and >= 128", (long long)k_row_stride);
-  if (num_pages > 1 && (k_page_stride <= 0 || k_page_stride % 8 != 0))
-    return fail(QSA_ERR_ALIGNMENT, "k_page_stride = %lld must be a positive multiple of 8", (long long)k_page_stride);
+  const int kb = fp8 ? 1 : 2;  // bytes per key element
+  const int64_t kmul = 16 / kb;
+  if (k_row_stride < 128 || k_row_stride % kmul != 0)
+    return fail(QSA_ERR_ALIGNMENT, "k_row_stride = %lld must be a multiple of %lld and >= 128",
+                (long long)k_row_stride, (long long)kmul);
+  if (num_pages > 1 && (k_page_stride <= 0 || k_page_stride % kmul != 0))
+    return fail(QSA_ERR_ALIGNMENT, "k_page_stride = %lld must be a positive multiple of %lld",
+                (long long)k_page_stride, (long long)kmul);
   if (max_pages > 0 && B > 1 && pt_stride < max_pages)
     return fail(QSA_ERR_INVALID_ARG, "pt_stride = %lld is below max_pages = %d", (long long)pt_stride, max_pages);
   if (Q > 1 && out_stride_t < W) return fail(QSA_ERR_INVALID_ARG, "out_stride_t is below W");
@@ -409,7 +419,7 @@ qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_
   {
     const Range ro = span(out, 4, B, B > 1 ? out_stride_b : 0, Q, Q > 1 ? out_stride_t : 0, 1, 0, W);
     const Range rq = span(q, 2, B, qs[0], Q, qs[1], 4, qs[2], 128);
-    const Range rk = span(k_cache, 2, num_pages, num_pages > 1 ? k_page_stride : 0, page_size, k_row_stride, 1, 0, 128);
+    const Range rk = span(k_cache, kb, num_pages, num_pages > 1 ? k_page_stride : 0, page_size, k_row_stride, 1, 0, 128);
     const Range rs = span(seq_lens, 4, B, 1, 1, 0, 1, 0, 1);
     bool bad = overlaps(ro, rq) || overlaps(ro, rk) || overlaps(ro, rs);
     if (max_pages > 0) bad = bad || overlaps(ro, span(page_table, 4, B, B > 1 ? pt_stride : 0, 1, 0, 1, 0, max_pages));
@@ -424,7 +434,8 @@ qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_
   p.q_sb = B > 1 ? q_stride_b : 0;
   p.q_st = Q > 1 ? q_stride_t : 0;
   p.q_sh = q_stride_h;
-  p.k_cache = static_cast<const uint16_t*>(k_cache);
+  p.k_cache = fp8 ? nullptr : static_cast<const uint16_t*>(k_cache);
+  p.k8 = fp8 ? static_cast<const uint8_t*>(k_cache) : nullptr;
   p.k_page_stride = num_pages > 1 ? k_page_stride : 0;
   p.k_row_stride = k_row_stride;
   p.num_pages = num_pages;
@@ -432,7 +443,7 @@ qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_
   p.max_pages = max_pages;
   p.Q = Q;
   p.log2_ps = page_size == 8 ? 3 : page_size == 16 ? 4 : page_size == 32 ? 5 : 6;
-  p.scale = scale;
+  p.scale = fp8 ? scale * k_scale : scale;
   p.out_sb = out_stride_b;
   p.out_st = out_stride_t;
   p.W = W;
@@ -443,12 +454,37 @@ qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_
     p.page_table = max_pages > 0 ? page_table + (int64_t)b0 * pt_stride : page_table;
     p.seq_lens = seq_lens + b0;
     p.out = out + (int64_t)b0 * out_stride_b;
-    qsa::decode::decode_kernel<<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES,
-                                 static_cast<cudaStream_t>(stream)>>>(p);
+    if (fp8)
+      qsa::decode::decode_kernel<true><<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES,
+                                         static_cast<cudaStream_t>(stream)>>>(p);
+    else
+      qsa::decode::decode_kernel<false><<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES,
+                                          static_cast<cudaStream_t>(stream)>>>(p);
     st = launch_status("decode kernel");
     if (st != QSA_OK) return st;
   }
   return ok();
+}
+
+qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
+                            const void* k_cache, int64_t num_pages, int32_t page_size, int64_t k_page_stride,
+                            int64_t k_row_stride, const int32_t* page_table, int64_t pt_stride, int32_t max_pages,
+                            const int32_t* seq_lens, int32_t B, int32_t Q, float scale, float* out,
+                            int64_t out_stride_b, int64_t out_stride_t, int32_t W, void* stream) {
+  return decode_common(q, q_stride_b, q_stride_t, q_stride_h, k_cache, false, 1.f, num_pages, page_size,
+                       k_page_stride, k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale, out,
+                       out_stride_b, out_stride_t, W, stream);
+}
+
+qsa_status_t qsa_mqa_decode_fp8(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
+                                const void* k_cache, float k_scale, int64_t num_pages, int32_t page_size,
+                                int64_t k_page_stride, int64_t k_row_stride, const int32_t* page_table,
+                                int64_t pt_stride, int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t Q,
+                                float scale, float* out, int64_t out_stride_b, int64_t out_stride_t, int32_t W,
+                                void* stream) {
+  return decode_common(q, q_stride_b, q_stride_t, q_stride_h, k_cache, true, k_scale, num_pages, page_size,
+                       k_page_stride, k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale, out,
+                       out_stride_b, out_stride_t, W, stream);
 }
 
 qsa_status_t qsa_mqa_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k, int64_t k_stride,

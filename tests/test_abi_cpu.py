@@ -76,6 +76,46 @@ def test_decode_empty_batch_is_a_no_op():
     assert decode(W=0)[0] == OK
 
 
+def decode_fp8(**kw):
+    a = dict(q=A, sb=2048, st=512, sh=128, k=A + S, kscale=0.01, pages=100, ps=64, kps=64 * 128, krs=128,
+             pt=A + 2 * S, pts=10, maxp=10, sl=A + 3 * S, B=4, Q=4, scale=0.088, out=A + 4 * S, osb=4 * 1000,
+             ost=1000, W=1000)
+    a.update(kw)
+    L = qsa.lib()
+    st = L.qsa_mqa_decode_fp8(a["q"], a["sb"], a["st"], a["sh"], a["k"], a["kscale"], a["pages"], a["ps"],
+                              a["kps"], a["krs"], a["pt"], a["pts"], a["maxp"], a["sl"], a["B"], a["Q"], a["scale"],
+                              a["out"], a["osb"], a["ost"], a["W"], None)
+    return st, L.qsa_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(kscale=0.0), INVALID), (dict(kscale=-0.5), INVALID), (dict(kscale=float("nan")), INVALID),
+    (dict(kscale=float("inf")), INVALID), (dict(kscale=1e30, scale=1e30), INVALID),
+    (dict(krs=136), ALIGN),            # 8-byte multiple: fine for bf16 elements, not for 1-byte codes
+    (dict(kps=64 * 128 + 8), ALIGN), (dict(krs=112), ALIGN), (dict(k=A + S + 8), ALIGN),
+    (dict(Q=5), UNSUP), (dict(ps=12), UNSUP), (dict(sh=100), ALIGN),
+    (dict(out=A + S + 64), INVALID),   # out overlaps the 1-byte cache
+])
+def test_decode_fp8_rejects(kw, code):
+    st, detail = decode_fp8(**kw)
+    assert st == code, detail
+    assert detail
+
+
+def test_decode_fp8_empty_batch_is_a_no_op():
+    assert decode_fp8(B=0)[0] == OK
+    assert decode_fp8(W=0)[0] == OK
+
+
+def test_decode_fp8_cache_span_uses_one_byte_elements():
+    # the bf16 span of this cache (100 pages x 16 KB) would reach out; the fp8 one (100 x 8 KB) does not
+    end8 = A + S + 100 * 64 * 128
+    st, detail = decode_fp8(out=end8 + 4096)     # passes validation (then needs a GPU)
+    assert st != INVALID and "overlap" not in detail, detail
+    st, detail = decode_fp8(out=end8 - 4096)
+    assert st == INVALID and "overlap" in detail, detail
+
+
 def prefill(**kw):
     a = dict(q=A, st=512, sh=128, k=A + S, ks_=128, Nk=1000, ks=A + 2 * S, ke=A + 3 * S, T=100, scale=0.088,
              out=A + 4 * S, os=2000, W=1000)

@@ -112,3 +112,109 @@ def test_decode_zero_queries_give_zero():
     d = wl.make_decode("zero", [800, 333], Q=4, page_size=64, seed=13)
     d.q = torch.zeros_like(d.q)
     run_case(d)
+
+
+# ---------------------------------------------------------------- fp8 E4M3 key cache
+
+def run_case_fp8(d: wl.DecodeInputs, codes=None, k_scale=None, q=None, W=None, kc_dev=None, out=None):
+    """The fp8 entry against the oracle's fp8 entry; the tolerance is the bf16
+    one on the dequantised keys (torch's E4M3 decoding times k_scale)."""
+    W = d.W if W is None else W
+    q = d.q if q is None else q
+    if codes is None:
+        codes, k_scale = wl.e4m3_cache(d.k_cache, k_scale)
+    dev = torch.device("cuda", 0)
+    res = qsa.mqa_decode_fp8(q.to(dev) if q.device.type == "cpu" else q,
+                             codes.to(dev) if kc_dev is None else kc_dev, k_scale,
+                             d.page_table.to(dev), d.seq_lens.to(dev), W, scale=SCALE, out=out)
+    torch.cuda.synchronize()
+    assert qsa.device_error() == 0
+    gpu = res.cpu().numpy()
+    ref = oracle.decode_fp8(q.cpu(), codes, k_scale, d.page_table, d.seq_lens, W, scale=SCALE)
+    kdq = codes.view(torch.float8_e4m3fn).to(torch.float64) * k_scale
+    loose, tight = decode_bounds(q.cpu(), kdq, d.page_table, W, SCALE)
+    return compare_scores(gpu, ref, loose, tight)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_decode_fp8_full_config(cfg):
+    """The three decode workloads at full size with the fp8 cache, every element."""
+    st = run_case_fp8(wl.make_config(cfg))
+    assert st["entries"] > 0
+
+
+@pytest.mark.parametrize("ps", [8, 16, 32, 64])
+@pytest.mark.parametrize("Q", [1, 2, 3, 4])
+def test_decode_fp8_ragged(ps, Q):
+    lens = [0, 1, 3, 4, 5, 7, 130, 511, 512, 513, 2049, 4 * 128 * 3 + 6]
+    d = wl.make_decode("ragged", lens, Q=Q, page_size=ps, seed=ps * 10 + Q + 500, W=max(lens) // 4 + 37)
+    run_case_fp8(d)
+
+
+def test_decode_fp8_invalid_pages_and_narrow_w():
+    d = wl.make_decode("bad_pages", [900, 1400, 333, 2000], Q=4, page_size=16, seed=17, table_pad=2)
+    t = d.page_table.clone()
+    P = d.k_cache.shape[0]
+    t[0, 1] = -1
+    t[1, 3] = P + 4
+    t[2, 0] = -7
+    t[3, 5:] = -1
+    d.page_table = t
+    run_case_fp8(d)
+    run_case_fp8(d, W=100)
+
+
+@pytest.mark.parametrize("k_scale", [2.0 ** -7, 0.0173, 1.0, 3.5])
+def test_decode_fp8_every_code(k_scale):
+    """Uniformly random finite codes: subnormals, both zeros and +-448 all occur."""
+    d = wl.make_decode("codes", [3000, 777, 64, 1500], Q=3, page_size=32, seed=19)
+    g = torch.Generator().manual_seed(20)
+    codes = torch.randint(0, 256, d.k_cache.shape, generator=g, dtype=torch.int32)
+    codes[(codes == 0x7F) | (codes == 0xFF)] = 0x7E
+    codes = codes.to(torch.uint8)
+    run_case_fp8(d, codes=codes, k_scale=k_scale)
+
+
+def test_decode_fp8_query_dynamic_range():
+    """Query rows far outside fp16's range, tiny rows, zero rows and rows that
+    mix magnitudes 2^20 apart (the kernel scales each row by a power of two)."""
+    d = wl.make_decode("qrange", [2000, 1000, 600, 3000], Q=4, page_size=64, seed=21)
+    q = d.q.float()
+    q[0, :, 0] *= 2.0 ** 40
+    q[0, :, 1] *= 2.0 ** -40
+    q[1, 0] = 0.0
+    q[1, 1, 2] = 0.0
+    q[2, :, 0, :64] *= 2.0 ** 10
+    q[2, :, 0, 64:] *= 2.0 ** -10
+    q[3, :, :, 5] = 60000.0
+    q[3, 2] *= 2.0 ** -100
+    run_case_fp8(d, q=q.to(torch.bfloat16))
+
+
+def test_decode_fp8_strided_views():
+    """A cache view with 144-byte rows and padded pages, and a padded out."""
+    d = wl.make_decode("strided", [777, 1500, 64], Q=3, page_size=32, seed=23)
+    codes, ks = wl.e4m3_cache(d.k_cache)
+    P, ps = codes.shape[:2]
+    big = torch.zeros(P, ps + 2, 1, 144, dtype=torch.uint8)
+    big[:, :ps, :, :128] = codes
+    dev = torch.device("cuda", 0)
+    kc = big.to(dev)[:, :ps, :, :128]
+    out = torch.full((d.B, d.Q, d.W + 9), 7.0, device=dev)[:, :, :d.W]
+    run_case_fp8(d, codes=codes, k_scale=ks, kc_dev=kc, out=out)
+
+
+def test_decode_fp8_agrees_with_bf16_kernel_on_exact_keys():
+    """With a power-of-two k_scale the dequantised keys are exact in bf16; the
+    fp8 kernel's scores then match the bf16 kernel's within fp32 rounding."""
+    d = wl.make_config(2)
+    codes, _ = wl.e4m3_cache(d.k_cache)
+    ks = 2.0 ** -6
+    kbf = (codes.view(torch.float8_e4m3fn).to(torch.float32) * ks).to(torch.bfloat16)
+    dev = torch.device("cuda", 0)
+    a = qsa.mqa_decode_fp8(d.q.to(dev), codes.to(dev), ks, d.page_table.to(dev), d.seq_lens.to(dev), d.W)
+    b = qsa.mqa_decode(d.q.to(dev), kbf.to(dev), d.page_table.to(dev), d.seq_lens.to(dev), d.W)
+    a, b = a.cpu().numpy(), b.cpu().numpy()
+    assert np.array_equal(np.isneginf(a), np.isneginf(b))
+    live = np.isfinite(b)
+    assert np.allclose(a[live], b[live], rtol=1e-5, atol=1e-5)

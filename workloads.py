@@ -155,6 +155,20 @@ def make_decode(name: str, seq_lens: list[int], Q: int, page_size: int, seed: in
                         meta={"seed": seed, "context_tokens": list(seq_lens)})
 
 
+def e4m3_cache(k_cache: torch.Tensor, k_scale: float | None = None) -> tuple[torch.Tensor, float]:
+    """An fp8 E4M3 copy of a bf16 key pool, as the cache writer stores it
+    (vLLM qsa_prepare.py, "_to_dst_dtype": the bf16 key divided by the cache
+    scale, converted to E4M3 by torch).  ``k_scale`` defaults to the pool's
+    largest magnitude / 448 (the largest finite E4M3 value), so no code
+    saturates and none is NaN.  Returns (uint8 codes of the same shape,
+    k_scale)."""
+    if k_scale is None:
+        amax = float(k_cache.float().abs().max()) if k_cache.numel() else 1.0
+        k_scale = amax / 448.0 if amax > 0 else 1.0
+    codes = (k_cache.float() / k_scale).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, float(k_scale)
+
+
 def make_prefill(name: str, new_tokens: list[int], prefixes: list[int], seed: int,
                  W: int | None = None) -> PrefillInputs:
     """Packed prefill inputs: sequence s has ``prefixes[s]`` cached tokens and

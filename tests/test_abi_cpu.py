@@ -181,6 +181,28 @@ def test_binding_refuses_cpu_tensors():
                        torch.zeros(1, dtype=torch.int32), 4)
 
 
+def test_fp8_binding_refuses_cpu_tensors_and_wrong_dtypes():
+    q = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
+    pt, sl = torch.zeros(1, 1, dtype=torch.int32), torch.zeros(1, dtype=torch.int32)
+    for kc in (torch.zeros(1, 16, 1, 128, dtype=torch.uint8),
+               torch.zeros(1, 16, 1, 128, dtype=torch.float8_e4m3fn),
+               torch.zeros(1, 16, 1, 128, dtype=torch.bfloat16)):
+        with pytest.raises(TypeError):
+            qsa.mqa_decode_fp8(q, kc, 0.5, pt, sl, 4)
+
+
+def test_oracle_fp8_accepts_float8_and_uint8_views():
+    import numpy as np
+    import oracle
+    import workloads as wl
+    d = wl.make_decode("views", [300, 77], Q=2, page_size=8, seed=3)
+    codes, ks = wl.e4m3_cache(d.k_cache)
+    a = oracle.decode_fp8(d.q, codes, ks, d.page_table, d.seq_lens, d.W, threads=1)
+    b = oracle.decode_fp8(d.q, codes.view(torch.float8_e4m3fn), ks, d.page_table, d.seq_lens, d.W, threads=1)
+    assert np.array_equal(a, b)
+    assert np.isfinite(a).any()
+
+
 def test_selftest_rejects_long_limit():
     L = qsa.lib()
     assert L.qsa_selftest_bounded_wait(20_000_000_000, 0, None) == INVALID, L.qsa_last_error_detail().decode()

@@ -218,3 +218,26 @@ def test_decode_fp8_agrees_with_bf16_kernel_on_exact_keys():
     assert np.array_equal(np.isneginf(a), np.isneginf(b))
     live = np.isfinite(b)
     assert np.allclose(a[live], b[live], rtol=1e-5, atol=1e-5)
+
+
+# ---------------------------------------------------------------- many requests
+
+def _many(B, Q, ps, seed, max_len=400):
+    g = np.random.default_rng(seed)
+    lens = g.integers(0, max_len + 1, size=B).tolist()
+    lens[0] = max_len                       # the widest row sets W
+    return wl.make_decode(f"many{B}", lens, Q=Q, page_size=ps, seed=seed)
+
+
+@pytest.mark.parametrize("B,Q,ps", [
+    (100, 2, 16),     # block-wide prefix scan, one chunk per warp over several 32-request groups
+    (1184, 1, 8),     # the largest batch with two warps per request
+    (1500, 3, 32),    # block-wide scan, warps take contiguous tile ranges across requests
+    (8200, 2, 8),     # more requests than one launch takes (two launches)
+])
+def test_decode_many_requests(B, Q, ps):
+    run_case(_many(B, Q, ps, seed=B + Q))
+
+
+def test_decode_fp8_many_requests():
+    run_case_fp8(_many(1500, 4, 16, seed=99))

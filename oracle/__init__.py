@@ -29,14 +29,16 @@ def _bind(L: C.CDLL) -> C.CDLL:
     L.qsa_oracle_decode_visible.argtypes = [_vp, _i64, _i64, _vp]
     L.qsa_oracle_prefill_intervals.argtypes = [_vp, _vp, _vp, _i64, _vp, _vp]
     L.qsa_oracle_decode.argtypes = [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _i64, _i64,
-                                    _vp, _i64, _i64, _vp, _i64, _i64, _f64, _vp, _i64, _int]
+                                    _vp, _i64, _i64, _vp, _i64, _i64, _f64, _vp, _i64, _int, _int]
     L.qsa_oracle_decode_entries.argtypes = [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _i64, _i64,
                                             _vp, _i64, _i64, _vp, _i64, _i64, _f64,
-                                            _vp, _vp, _vp, _i64, _vp, _int]
+                                            _vp, _vp, _vp, _i64, _vp, _int, _int]
     L.qsa_oracle_prefill.argtypes = [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f64,
-                                     _vp, _i64, _int]
+                                     _vp, _i64, _int, _int]
     L.qsa_oracle_prefill_entries.argtypes = [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _f64,
-                                             _vp, _vp, _i64, _vp, _int]
+                                             _vp, _vp, _i64, _vp, _int, _int]
+    L.qsa_oracle_f16_to_double.argtypes = [C.c_uint16]
+    L.qsa_oracle_f16_to_double.restype = C.c_double
     L.qsa_oracle_topk.argtypes = [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _int]
     L.qsa_oracle_e4m3_to_double.argtypes = [C.c_uint8]
     L.qsa_oracle_e4m3_to_double.restype = C.c_double
@@ -49,17 +51,27 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(C.c_void_p)
 
 
-def _bf16_bits(x) -> tuple[np.ndarray, tuple[int, ...]]:
-    """bf16 tensor/array -> (uint16 bit array, element strides)."""
-    if hasattr(x, "view") and hasattr(x, "dtype") and str(x.dtype) == "torch.bfloat16":
+def _bits16(x) -> tuple[np.ndarray, tuple[int, ...], int]:
+    """bf16 / fp16 tensor, or a uint16 array of bf16 bits -> (uint16 bit
+    array, element strides, 1 if fp16 else 0)."""
+    if hasattr(x, "view") and hasattr(x, "dtype") and str(x.dtype) in ("torch.bfloat16", "torch.float16"):
         import torch
+        f16 = int(x.dtype == torch.float16)
         x = x.detach().cpu()
         bits = x.view(torch.int16).numpy().view(np.uint16)
-        return bits, tuple(x.stride())
+        return bits, tuple(x.stride()), f16
     a = np.asarray(x)
     if a.dtype != np.uint16:
-        raise TypeError("bf16 data must be a torch.bfloat16 tensor or uint16 bit array")
-    return a, tuple(s // 2 for s in a.strides)
+        raise TypeError("16-bit data must be a torch.bfloat16 / torch.float16 tensor or a uint16 bf16 bit array")
+    return a, tuple(s // 2 for s in a.strides), 0
+
+
+def _bf16_bits(x) -> tuple[np.ndarray, tuple[int, ...]]:
+    """bf16 tensor/array -> (uint16 bit array, element strides)."""
+    bits, strides, f16 = _bits16(x)
+    if f16:
+        raise TypeError("expected bf16 data")
+    return bits, strides
 
 
 def _i32(x) -> np.ndarray:
@@ -101,25 +113,32 @@ class Oracle:
 
     @staticmethod
     def _decode_common(q, k_cache, page_table, seq_lens):
-        qb, qs = _bf16_bits(q)
-        kb, kst = _bf16_bits(k_cache)
+        qb, qs, f16 = _bits16(q)
+        kb, kst, kf16 = _bits16(k_cache)
+        if f16 != kf16:
+            raise TypeError("q and k_cache must have the same dtype (bf16 or fp16)")
         if len(qs) != 4 or qs[3] != 1:
             raise ValueError("q must be [B, Q, 4, 128] with unit feature stride")
         if len(kst) != 4 or kst[3] != 1:
             raise ValueError("k_cache must be [pages, page_size, 1, 128] with unit feature stride")
-        return qb, qs, kb, kst, _i32(page_table), _i32(seq_lens)
+        return qb, qs, kb, kst, _i32(page_table), _i32(seq_lens), f16
 
     def decode(self, q, k_cache, page_table, seq_lens, W: int, scale: float = SCALE,
                threads: int = 0) -> np.ndarray:
-        """fp64 scores [B, Q, W] of the paged decode / spec-decode path."""
-        qb, qs, kb, kst, pt, sl = self._decode_common(q, k_cache, page_table, seq_lens)
+        """fp64 scores [B, Q, W] of the paged decode / spec-decode path (q and
+        k_cache both bf16 or both fp16)."""
+        qb, qs, kb, kst, pt, sl, f16 = self._decode_common(q, k_cache, page_table, seq_lens)
         B, Q = qb.shape[0], qb.shape[1]
         out = np.empty((B, Q, W), dtype=np.float64)
         self.L.qsa_oracle_decode(_ptr(qb), qs[0], qs[1], qs[2], _ptr(kb), kb.shape[0],
                                  kb.shape[1], kst[0], kst[1], _ptr(pt), pt.shape[1],
                                  pt.shape[1], _ptr(sl), B, Q, float(scale), _ptr(out), W,
-                                 threads)
+                                 threads, f16)
         return out
+
+    def f16_to_double(self, bits: int) -> float:
+        """Value of one fp16 bit pattern."""
+        return float(self.L.qsa_oracle_f16_to_double(int(bits) & 0xFFFF))
 
     def e4m3_to_double(self, code: int) -> float:
         """Value of one fp8 E4M3 code."""
@@ -155,7 +174,7 @@ class Oracle:
     def decode_entries(self, q, k_cache, page_table, seq_lens, b, i, n, scale: float = SCALE,
                        threads: int = 0) -> np.ndarray:
         """fp64 scores of the listed decode entries (row (b[e], i[e]), column n[e])."""
-        qb, qs, kb, kst, pt, sl = self._decode_common(q, k_cache, page_table, seq_lens)
+        qb, qs, kb, kst, pt, sl, f16 = self._decode_common(q, k_cache, page_table, seq_lens)
         bb = np.ascontiguousarray(b, dtype=np.int64)
         ii = np.ascontiguousarray(i, dtype=np.int64)
         nn = np.ascontiguousarray(n, dtype=np.int64)
@@ -164,38 +183,41 @@ class Oracle:
                                          kb.shape[1], kst[0], kst[1], _ptr(pt), pt.shape[1],
                                          pt.shape[1], _ptr(sl), qb.shape[0], qb.shape[1],
                                          float(scale), _ptr(bb), _ptr(ii), _ptr(nn),
-                                         bb.shape[0], _ptr(out), threads)
+                                         bb.shape[0], _ptr(out), threads, f16)
         return out
 
     @staticmethod
     def _prefill_common(q, k, ks, ke):
-        qb, qs = _bf16_bits(q)
-        kb, kst = _bf16_bits(k)
+        qb, qs, f16 = _bits16(q)
+        kb, kst, kf16 = _bits16(k)
+        if f16 != kf16:
+            raise TypeError("q and k must have the same dtype (bf16 or fp16)")
         if len(qs) != 3 or qs[2] != 1:
             raise ValueError("q must be [T, 4, 128] with unit feature stride")
         if len(kst) != 2 or kst[1] != 1:
             raise ValueError("k must be [Nk, 128] with unit feature stride")
-        return qb, qs, kb, kst, _i32(ks), _i32(ke)
+        return qb, qs, kb, kst, _i32(ks), _i32(ke), f16
 
     def prefill(self, q, k, ks, ke, W: int, scale: float = SCALE, threads: int = 0) -> np.ndarray:
-        """fp64 scores [T, W] of the packed prefill path (column j holds key ks[t] + j)."""
-        qb, qs, kb, kst, a, b = self._prefill_common(q, k, ks, ke)
+        """fp64 scores [T, W] of the packed prefill path (column j holds key ks[t] + j;
+        q and k both bf16 or both fp16)."""
+        qb, qs, kb, kst, a, b, f16 = self._prefill_common(q, k, ks, ke)
         T = qb.shape[0]
         out = np.empty((T, W), dtype=np.float64)
         self.L.qsa_oracle_prefill(_ptr(qb), qs[0], qs[1], _ptr(kb), kst[0], kb.shape[0],
-                                  _ptr(a), _ptr(b), T, float(scale), _ptr(out), W, threads)
+                                  _ptr(a), _ptr(b), T, float(scale), _ptr(out), W, threads, f16)
         return out
 
     def prefill_entries(self, q, k, ks, ke, t, j, scale: float = SCALE,
                         threads: int = 0) -> np.ndarray:
         """fp64 scores of the listed prefill entries (row t[e], column j[e])."""
-        qb, qs, kb, kst, a, b = self._prefill_common(q, k, ks, ke)
+        qb, qs, kb, kst, a, b, f16 = self._prefill_common(q, k, ks, ke)
         tt = np.ascontiguousarray(t, dtype=np.int64)
         jj = np.ascontiguousarray(j, dtype=np.int64)
         out = np.empty(tt.shape[0], dtype=np.float64)
         self.L.qsa_oracle_prefill_entries(_ptr(qb), qs[0], qs[1], _ptr(kb), kst[0],
                                           kb.shape[0], _ptr(a), _ptr(b), float(scale),
-                                          _ptr(tt), _ptr(jj), tt.shape[0], _ptr(out), threads)
+                                          _ptr(tt), _ptr(jj), tt.shape[0], _ptr(out), threads, f16)
         return out
 
     def topk(self, scores, lengths, k: int, threads: int = 0) -> np.ndarray:

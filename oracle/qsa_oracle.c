@@ -50,6 +50,25 @@ static double bf16_to_double(uint16_t bits) {
     return (double)f;
 }
 
+/* Value of an IEEE binary16 (fp16) bit pattern: 1 sign bit, 5 exponent bits
+ * with bias 15, 10 mantissa bits; exponent 0 holds zero and the subnormals
+ * m * 2^-24, exponent 31 holds the infinities and NaNs. */
+static double f16_to_double(uint16_t bits) {
+    int sign = bits >> 15, ex = (bits >> 10) & 31, man = bits & 1023;
+    double mag;
+    if (ex == 31) mag = man ? NAN : INFINITY;
+    else if (ex == 0) mag = ldexp((double)man, -24);
+    else mag = ldexp(1.0 + man / 1024.0, ex - 15);
+    return sign ? -mag : mag;
+}
+
+double qsa_oracle_f16_to_double(uint16_t bits) { return f16_to_double(bits); }
+
+/* A 16-bit input element: bf16 or (f16 != 0) fp16. */
+static double elem_to_double(uint16_t bits, int f16) {
+    return f16 ? f16_to_double(bits) : bf16_to_double(bits);
+}
+
 static int64_t floor_div(int64_t a, int64_t b) {
     int64_t q = a / b;
     if ((a % b != 0) && ((a < 0) != (b < 0))) q -= 1;
@@ -146,8 +165,8 @@ double qsa_oracle_e4m3_to_double(uint8_t code) {
  * cache's dequantisation scale k_scale (the cache stores e4m3(bf16(k) /
  * k_scale): vLLM qsa_prepare.py, "_to_dst_dtype", rounds to bf16 first, then
  * scales for an fp8 destination). */
-static void key_row_bf16(const uint16_t *k_row, double *k) {
-    for (int e = 0; e < QSA_DIM; ++e) k[e] = bf16_to_double(k_row[e]);
+static void key_row_16(const uint16_t *k_row, int f16, double *k) {
+    for (int e = 0; e < QSA_DIM; ++e) k[e] = elem_to_double(k_row[e], f16);
 }
 
 static void key_row_e4m3(const uint8_t *k_row, double k_scale, double *k) {
@@ -155,13 +174,13 @@ static void key_row_e4m3(const uint8_t *k_row, double k_scale, double *k) {
 }
 
 /* scale * sum_h max(0, q_h . k) for one query row (4 heads) and one key. */
-static double head_sum_score(const uint16_t *q_row, int64_t q_stride_h,
+static double head_sum_score(const uint16_t *q_row, int64_t q_stride_h, int f16,
                              const double *k, double scale) {
     double s = 0.0;
     for (int h = 0; h < QSA_HEADS; ++h) {
         const uint16_t *qh = q_row + h * q_stride_h;
         double d = 0.0;
-        for (int c = 0; c < QSA_DIM; ++c) d += bf16_to_double(qh[c]) * k[c];
+        for (int c = 0; c < QSA_DIM; ++c) d += elem_to_double(qh[c], f16) * k[c];
         s += d > 0.0 ? d : 0.0;
     }
     return scale * s;
@@ -174,6 +193,7 @@ typedef struct {
     const int32_t *seq_lens; int64_t B, Q;
     double scale;
     const uint8_t *k8; double k_scale;   /* fp8 cache when k8 != NULL (then k_cache is unused) */
+    int f16;                             /* q (and a 16-bit cache) hold fp16 instead of bf16 */
 } decode_args;
 
 /* Score of decode row (b, i) against compressed key n, or -inf when masked. */
@@ -189,8 +209,8 @@ static double decode_entry(const decode_args *a, int64_t b, int64_t i, int64_t n
     int64_t row_off = page * a->k_page_stride + (n % a->page_size) * a->k_row_stride;
     double k[QSA_DIM];
     if (a->k8) key_row_e4m3(a->k8 + row_off, a->k_scale, k);
-    else key_row_bf16(a->k_cache + row_off, k);
-    return head_sum_score(q_row, a->q_sh, k, a->scale);
+    else key_row_16(a->k_cache + row_off, a->f16, k);
+    return head_sum_score(q_row, a->q_sh, a->f16, k, a->scale);
 }
 
 typedef struct { decode_args a; double *out; int64_t W; } decode_full_ctx;
@@ -203,16 +223,17 @@ static void decode_rows(void *vctx, int64_t begin, int64_t end) {
     }
 }
 
-/* out[(b * Q + i) * W + n] for every row and every n < W. */
+/* out[(b * Q + i) * W + n] for every row and every n < W; q and k_cache
+ * hold bf16, or fp16 when f16 != 0. */
 void qsa_oracle_decode(const uint16_t *q, int64_t q_sb, int64_t q_st, int64_t q_sh,
                        const uint16_t *k_cache, int64_t num_pages, int64_t page_size,
                        int64_t k_page_stride, int64_t k_row_stride,
                        const int32_t *page_table, int64_t pt_stride, int64_t max_pages,
                        const int32_t *seq_lens, int64_t B, int64_t Q, double scale,
-                       double *out, int64_t W, int nthreads) {
+                       double *out, int64_t W, int nthreads, int f16) {
     decode_full_ctx c = {{q, q_sb, q_st, q_sh, k_cache, num_pages, page_size, k_page_stride,
                           k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale,
-                          NULL, 0.0},
+                          NULL, 0.0, f16},
                          out, W};
     parallel_for(B * Q, nthreads, decode_rows, &c);
 }
@@ -227,7 +248,7 @@ void qsa_oracle_decode_fp8(const uint16_t *q, int64_t q_sb, int64_t q_st, int64_
                            double *out, int64_t W, int nthreads) {
     decode_full_ctx c = {{q, q_sb, q_st, q_sh, NULL, num_pages, page_size, k_page_stride,
                           k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale,
-                          k8, k_scale},
+                          k8, k_scale, 0},
                          out, W};
     parallel_for(B * Q, nthreads, decode_rows, &c);
 }
@@ -246,10 +267,10 @@ void qsa_oracle_decode_entries(const uint16_t *q, int64_t q_sb, int64_t q_st, in
                                const int32_t *page_table, int64_t pt_stride, int64_t max_pages,
                                const int32_t *seq_lens, int64_t B, int64_t Q, double scale,
                                const int64_t *bb, const int64_t *ii, const int64_t *nn,
-                               int64_t count, double *out, int nthreads) {
+                               int64_t count, double *out, int nthreads, int f16) {
     decode_entries_ctx c = {{q, q_sb, q_st, q_sh, k_cache, num_pages, page_size, k_page_stride,
                              k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale,
-                             NULL, 0.0},
+                             NULL, 0.0, f16},
                             bb, ii, nn, out};
     parallel_for(count, nthreads, decode_entries_range, &c);
 }
@@ -259,6 +280,7 @@ typedef struct {
     const uint16_t *k; int64_t k_stride, Nk;
     const int32_t *ks, *ke;
     double scale;
+    int f16;   /* q and k hold fp16 instead of bf16 */
 } prefill_args;
 
 /* Score of prefill row t at column j (key ks[t] + j), or -inf when masked. */
@@ -268,8 +290,8 @@ static double prefill_entry(const prefill_args *a, int64_t t, int64_t j) {
     int64_t n = (int64_t)a->ks[t] + j;
     if (j < 0 || n < lo || n >= hi) return -INFINITY;
     double k[QSA_DIM];
-    key_row_bf16(a->k + n * a->k_stride, k);
-    return head_sum_score(a->q + t * a->q_st, a->q_sh, k, a->scale);
+    key_row_16(a->k + n * a->k_stride, a->f16, k);
+    return head_sum_score(a->q + t * a->q_st, a->q_sh, a->f16, k, a->scale);
 }
 
 typedef struct { prefill_args a; double *out; int64_t W; } prefill_full_ctx;
@@ -280,12 +302,13 @@ static void prefill_rows(void *vctx, int64_t begin, int64_t end) {
         for (int64_t j = 0; j < c->W; ++j) c->out[t * c->W + j] = prefill_entry(&c->a, t, j);
 }
 
-/* out[t * W + j] for every row t < T and column j < W. */
+/* out[t * W + j] for every row t < T and column j < W; q and k hold bf16,
+ * or fp16 when f16 != 0. */
 void qsa_oracle_prefill(const uint16_t *q, int64_t q_st, int64_t q_sh,
                         const uint16_t *k, int64_t k_stride, int64_t Nk,
                         const int32_t *ks, const int32_t *ke, int64_t T, double scale,
-                        double *out, int64_t W, int nthreads) {
-    prefill_full_ctx c = {{q, q_st, q_sh, k, k_stride, Nk, ks, ke, scale}, out, W};
+                        double *out, int64_t W, int nthreads, int f16) {
+    prefill_full_ctx c = {{q, q_st, q_sh, k, k_stride, Nk, ks, ke, scale, f16}, out, W};
     parallel_for(T, nthreads, prefill_rows, &c);
 }
 
@@ -301,8 +324,8 @@ void qsa_oracle_prefill_entries(const uint16_t *q, int64_t q_st, int64_t q_sh,
                                 const uint16_t *k, int64_t k_stride, int64_t Nk,
                                 const int32_t *ks, const int32_t *ke, double scale,
                                 const int64_t *tt, const int64_t *jj, int64_t count,
-                                double *out, int nthreads) {
-    prefill_entries_ctx c = {{q, q_st, q_sh, k, k_stride, Nk, ks, ke, scale}, tt, jj, out};
+                                double *out, int nthreads, int f16) {
+    prefill_entries_ctx c = {{q, q_st, q_sh, k, k_stride, Nk, ks, ke, scale, f16}, tt, jj, out};
     parallel_for(count, nthreads, prefill_entries_range, &c);
 }
 

@@ -19,7 +19,10 @@ when the oracle disagrees with:
   cache dtypes; vLLM qsa_prepare.py, "_to_dst_dtype"): torch's own E4M3
   decoding of all 256 codes and the format's fixed values, exact integer
   brute force with keys that E4M3 holds exactly, and the bf16 entry on keys
-  dequantised by torch.
+  dequantised by torch;
+* for fp16 inputs (the QSA docs' second input dtype, section "MQA score"):
+  torch's decoding of all 65,536 fp16 patterns, the bf16 entries on values
+  both formats hold exactly, and a closed form on a value only fp16 holds.
 
 The same functions run against deliberately broken builds of the oracle
 (``test_oracle_mutants.py``) to show that each plausible mistake trips a pin.
@@ -425,6 +428,54 @@ def pin_fp8_matches_bf16_on_dequantised_keys(orc):
     assert np.isfinite(got).sum() > 0
 
 
+# ---------------------------------------------------------------- fp16 inputs
+
+def pin_f16_decoder(orc):
+    """Every fp16 bit pattern against torch's float16 decoding (zeros of
+    both signs, subnormals down to 2^-24, the largest finite 65504,
+    infinities, NaNs)."""
+    bits = torch.arange(65536, dtype=torch.int32).to(torch.int16)
+    ref = bits.view(torch.float16).to(torch.float64).numpy()
+    got = np.array([orc.f16_to_double(b) for b in range(65536)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert got[0x0001] == 2.0 ** -24 and got[0x7BFF] == 65504.0 and got[0x3C00] == 1.0
+    assert got[0x7C00] == np.inf and got[0xFC00] == -np.inf
+    assert math.copysign(1.0, got[0x8000]) == -1.0
+
+
+def pin_f16_matches_bf16_on_shared_values(orc):
+    """Small integers are exact in both formats: the fp16 decode and prefill
+    entries must equal the bf16 ones on them, element for element."""
+    rng = np.random.default_rng(21)
+    q, kc, table, sl, W = paged_case(rng, 3, 4, 16, [300, 41, 130])
+    a = orc.decode(q, kc, table, sl, W, threads=2)
+    b = orc.decode(q.to(torch.float16), kc.to(torch.float16), table, sl, W, threads=2)
+    assert np.array_equal(a, b) and np.isfinite(a).sum() > 0
+    qp, kp, cu, total, offs, maxk = packed_case(rng, [9, 5], [30, 0])
+    ks, ke = orc.prefill_intervals(cu, total, offs)
+    a = orc.prefill(qp, kp, ks, ke, maxk + 2, threads=2)
+    b = orc.prefill(qp.to(torch.float16), kp.to(torch.float16), ks, ke, maxk + 2, threads=2)
+    assert np.array_equal(a, b) and np.isfinite(a).sum() > 0
+
+
+def pin_f16_closed_form(orc):
+    """q_0 = (1 + 2^-10) e_0 (exact in fp16, not in bf16) and k = e_0:
+    the score is exactly scale * (1 + 2^-10), and 0 with -q."""
+    q = torch.zeros(1, 4, 128, dtype=torch.float16)
+    q[0, 0, 0] = 1.0 + 2.0 ** -10
+    k = torch.zeros(1, 128, dtype=torch.float16)
+    k[0, 0] = 1.0
+    ks, ke = np.array([0], dtype=np.int32), np.array([1], dtype=np.int32)
+    got = orc.prefill(q, k, ks, ke, 1, scale=0.5)
+    assert got[0, 0] == 0.5 * (1.0 + 2.0 ** -10)
+    assert orc.prefill(-q, k, ks, ke, 1, scale=0.5)[0, 0] == 0.0
+    d = orc.decode(q.view(1, 1, 4, 128), k.view(1, 1, 1, 128).expand(1, 8, 1, 128).contiguous(),
+                   torch.zeros(1, 1, dtype=torch.int32), torch.tensor([4], dtype=torch.int32), 1, scale=0.5)
+    assert d[0, 0, 0] == 0.5 * (1.0 + 2.0 ** -10)
+
+
 ALL_PINS = [
     pin_visible_blocks_follow_cache_writer,
     pin_decode_positions_are_last_tokens,
@@ -440,4 +491,7 @@ ALL_PINS = [
     pin_e4m3_decoder,
     pin_fp8_decode_exact_bruteforce,
     pin_fp8_matches_bf16_on_dequantised_keys,
+    pin_f16_decoder,
+    pin_f16_matches_bf16_on_shared_values,
+    pin_f16_closed_form,
 ]

@@ -38,6 +38,12 @@ MUTANTS = {
     "e4m3 subnormals read as normals": ("if (e == 0) v = ldexp((double)m, -9);",
                                         "if (e == 0) v = ldexp(1.0 + m / 8.0, -7);"),
     "e4m3 sign ignored": ("return sign ? -v : v;", "return v;"),
+    "fp16 read as bf16": ("return f16 ? f16_to_double(bits) : bf16_to_double(bits);",
+                          "return bf16_to_double(bits);"),
+    "fp16 exponent bias off by one": ("else mag = ldexp(1.0 + man / 1024.0, ex - 15);",
+                                      "else mag = ldexp(1.0 + man / 1024.0, ex - 14);"),
+    "fp16 subnormals flushed": ("else if (ex == 0) mag = ldexp((double)man, -24);",
+                                "else if (ex == 0) mag = 0.0;"),
     "top-k keeps the smallest": ("if (a->v > b->v) return -1;\n    if (a->v < b->v) return 1;",
                                  "if (a->v < b->v) return -1;\n    if (a->v > b->v) return 1;"),
 }

@@ -363,6 +363,40 @@ def pin_topk_ties_and_padding(orc):
     assert orc.topk(s2, np.array([4], dtype=np.int32), 3)[0].tolist() == [1, 3, -1]
 
 
+def _repage(kc, table, B, ps2):
+    """The requests' keys laid out again with ps2 rows per page (pages in
+    reverse order in the pool, -1 past each request's pages)."""
+    keys = [torch.cat([kc[p, :, 0, :] for p in table[b].tolist() if p >= 0]) for b in range(B)]
+    pool, rows = [], []
+    for b in range(B):
+        kb = keys[b]
+        kb = torch.cat([kb, torch.zeros((-kb.shape[0]) % ps2, 128, dtype=kb.dtype)])
+        rows.append([])
+        for j in range(kb.shape[0] // ps2):
+            rows[b].append(len(pool))
+            pool.append(kb[j * ps2:(j + 1) * ps2])
+    n = len(pool)
+    width = max(len(r) for r in rows) + 1
+    t = np.full((B, width), -1, dtype=np.int32)
+    for b in range(B):
+        t[b, :len(rows[b])] = [n - 1 - p for p in rows[b]]
+    kc2 = torch.stack(pool[::-1])[:, :, None, :]
+    return kc2, torch.from_numpy(t)
+
+
+def pin_page_sizes_not_powers_of_two(orc):
+    """The production page size 196 (and 12) lays out the same keys: the
+    scores must not change, including blocks that straddle page edges."""
+    rng = np.random.default_rng(6)
+    B, Q, lens = 2, 3, [2000, 900]
+    q, kc, table, sl, W = paged_case(rng, B, Q, 8, lens, bad_pages=False)
+    ref = orc.decode(q, kc, table, sl, W)
+    for ps2 in (196, 12, 64):
+        kc2, t2 = _repage(kc, table, B, ps2)
+        assert np.array_equal(orc.decode(q, kc2, t2, sl, W), ref), ps2
+    assert np.isfinite(ref).sum() > 600
+
+
 # ---------------------------------------------------------------- fp8 cache
 
 def pin_e4m3_decoder(orc):
@@ -486,6 +520,7 @@ ALL_PINS = [
     pin_closed_forms,
     pin_invariants,
     pin_cross_entry_identities,
+    pin_page_sizes_not_powers_of_two,
     pin_topk_against_full_sort,
     pin_topk_ties_and_padding,
     pin_e4m3_decoder,

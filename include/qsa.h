@@ -111,6 +111,9 @@ qsa_status_t qsa_selftest_bounded_wait(uint64_t timeout_ns, int32_t arrive, void
  *              every n < W (columns past the visible keys are filled with
  *              -inf).  W >= max visible is the caller's choice; keys at
  *              n >= W are not scored.  out must not overlap any input.
+ *              Limit: min(B, 8192) * ceil(W / 8) must stay below 2^32 (the
+ *              kernel counts 8-key tiles in 32 bits; reaching it takes an
+ *              output of more than 128 GB); it is not checked.
  */
 qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
                             const void* k_cache, int64_t num_pages, int32_t page_size, int64_t k_page_stride,

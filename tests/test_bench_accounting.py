@@ -75,3 +75,13 @@ def test_source_digest_ignores_comments_and_blank_space(tmp_path, monkeypatch):
     assert bench.source_hash() == base
     f.write_text(text.replace("constexpr int BATCH = 4;", "constexpr int BATCH = 2;", 1))
     assert bench.source_hash() != base
+
+
+def test_fp8_decode_bytes_count_one_byte_per_key_element():
+    ctx = [1536, 10240, 43876, 7]
+    keys = sum(L // 4 for L in ctx)
+    for dql in (1, 4):
+        bf16 = bench.decode_bytes(ctx, dql)
+        fp8 = bench.decode_bytes(ctx, dql, 128)
+        assert bf16 - fp8 == keys * 128
+        assert fp8 == keys * 128 + dql * keys * 4 + len(ctx) * dql * 1024

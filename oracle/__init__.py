@@ -30,9 +30,6 @@ def _bind(L: C.CDLL) -> C.CDLL:
     L.qsa_oracle_prefill_intervals.argtypes = [_vp, _vp, _vp, _i64, _vp, _vp]
     L.qsa_oracle_decode.argtypes = [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _i64, _i64,
                                     _vp, _i64, _i64, _vp, _i64, _i64, _f64, _vp, _i64, _int, _int]
-    L.qsa_oracle_decode_entries.argtypes = [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _i64, _i64,
-                                            _vp, _i64, _i64, _vp, _i64, _i64, _f64,
-                                            _vp, _vp, _vp, _i64, _vp, _int, _int]
     L.qsa_oracle_prefill.argtypes = [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f64,
                                      _vp, _i64, _int, _int]
     L.qsa_oracle_prefill_entries.argtypes = [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _f64,
@@ -169,21 +166,6 @@ class Oracle:
         self.L.qsa_oracle_decode_fp8(_ptr(qb), qs[0], qs[1], qs[2], _ptr(kb), float(k_scale), kb.shape[0],
                                      kb.shape[1], kst[0], kst[1], _ptr(pt), pt.shape[1], pt.shape[1],
                                      _ptr(sl), B, Q, float(scale), _ptr(out), W, threads)
-        return out
-
-    def decode_entries(self, q, k_cache, page_table, seq_lens, b, i, n, scale: float = SCALE,
-                       threads: int = 0) -> np.ndarray:
-        """fp64 scores of the listed decode entries (row (b[e], i[e]), column n[e])."""
-        qb, qs, kb, kst, pt, sl, f16 = self._decode_common(q, k_cache, page_table, seq_lens)
-        bb = np.ascontiguousarray(b, dtype=np.int64)
-        ii = np.ascontiguousarray(i, dtype=np.int64)
-        nn = np.ascontiguousarray(n, dtype=np.int64)
-        out = np.empty(bb.shape[0], dtype=np.float64)
-        self.L.qsa_oracle_decode_entries(_ptr(qb), qs[0], qs[1], qs[2], _ptr(kb), kb.shape[0],
-                                         kb.shape[1], kst[0], kst[1], _ptr(pt), pt.shape[1],
-                                         pt.shape[1], _ptr(sl), qb.shape[0], qb.shape[1],
-                                         float(scale), _ptr(bb), _ptr(ii), _ptr(nn),
-                                         bb.shape[0], _ptr(out), threads, f16)
         return out
 
     @staticmethod

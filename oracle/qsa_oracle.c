@@ -253,28 +253,6 @@ void qsa_oracle_decode_fp8(const uint16_t *q, int64_t q_sb, int64_t q_st, int64_
     parallel_for(B * Q, nthreads, decode_rows, &c);
 }
 
-typedef struct { decode_args a; const int64_t *bb, *ii, *nn; double *out; } decode_entries_ctx;
-
-static void decode_entries_range(void *vctx, int64_t begin, int64_t end) {
-    decode_entries_ctx *c = (decode_entries_ctx *)vctx;
-    for (int64_t e = begin; e < end; ++e) c->out[e] = decode_entry(&c->a, c->bb[e], c->ii[e], c->nn[e]);
-}
-
-/* out[e] = score of decode row (bb[e], ii[e]) at column nn[e]. */
-void qsa_oracle_decode_entries(const uint16_t *q, int64_t q_sb, int64_t q_st, int64_t q_sh,
-                               const uint16_t *k_cache, int64_t num_pages, int64_t page_size,
-                               int64_t k_page_stride, int64_t k_row_stride,
-                               const int32_t *page_table, int64_t pt_stride, int64_t max_pages,
-                               const int32_t *seq_lens, int64_t B, int64_t Q, double scale,
-                               const int64_t *bb, const int64_t *ii, const int64_t *nn,
-                               int64_t count, double *out, int nthreads, int f16) {
-    decode_entries_ctx c = {{q, q_sb, q_st, q_sh, k_cache, num_pages, page_size, k_page_stride,
-                             k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale,
-                             NULL, 0.0, f16},
-                            bb, ii, nn, out};
-    parallel_for(count, nthreads, decode_entries_range, &c);
-}
-
 typedef struct {
     const uint16_t *q; int64_t q_st, q_sh;
     const uint16_t *k; int64_t k_stride, Nk;

@@ -233,6 +233,34 @@ def pin_prefill_exact_bruteforce(orc):
             assert got2[t, j] == want_tj, (t, j)
 
 
+def pin_prefill_entries_match_bruteforce(orc):
+    """The listed-entries form of the prefill oracle (the checker of the
+    full-size parity tests, which sample rows and columns) against exact
+    integer brute force: entries in shuffled order, repeated entries,
+    intervals that start below 0, end past the keys, are empty or reversed,
+    and columns past each interval."""
+    rng = np.random.default_rng(11)
+    new, pre = [6, 3, 9], [5, 0, 22]
+    q, k, _, _, _, _ = packed_case(rng, new, pre)
+    T, Nk = q.shape[0], k.shape[0]
+    ks = rng.integers(-4, Nk, size=T).astype(np.int32)
+    ke = (ks + rng.integers(-2, 12, size=T)).astype(np.int32)
+    ke[0], ks[1], ke[1], ks[2], ke[2] = Nk + 5, -3, 4, 3, 3
+    tt, jj = np.meshgrid(np.arange(T), np.arange(T), indexing="ij")
+    tt, jj = tt.ravel(), jj.ravel()
+    order = rng.permutation(tt.size)
+    tt = np.concatenate([tt[order], tt[order[:7]]])
+    jj = np.concatenate([jj[order], jj[order[:7]]])
+    got = orc.prefill_entries(q, k, ks, ke, tt, jj, scale=1.0, threads=3)
+    qi, ki = as_int(q), as_int(k)
+    for e in range(tt.size):
+        t, j = int(tt[e]), int(jj[e])
+        n = int(ks[t]) + j
+        ok = max(int(ks[t]), 0) <= n < min(int(ke[t]), Nk)
+        want = int_score(qi[t], ki[n]) if ok else -np.inf
+        assert got[e] == want, (e, t, j)
+
+
 def pin_closed_forms(orc):
     T = 3
     q = torch.zeros(T, 4, 128, dtype=torch.bfloat16)
@@ -517,6 +545,7 @@ ALL_PINS = [
     pin_prefill_intervals_follow_cache_writer,
     pin_decode_exact_bruteforce,
     pin_prefill_exact_bruteforce,
+    pin_prefill_entries_match_bruteforce,
     pin_closed_forms,
     pin_invariants,
     pin_cross_entry_identities,

@@ -26,6 +26,9 @@ MUTANTS = {
     "rows and requests transposed": ("int64_t b = r / c->a.Q, i = r % c->a.Q;",
                                      "int64_t b = r % c->a.B, i = r / c->a.B;"),
     "prefill columns absolute": ("int64_t n = (int64_t)a->ks[t] + j;", "int64_t n = j;"),
+    "prefill entries read row and column swapped": (
+        "c->out[e] = prefill_entry(&c->a, c->tt[e], c->jj[e]);",
+        "c->out[e] = prefill_entry(&c->a, c->jj[e], c->tt[e]);"),
     "prefill end not clipped to the interval": (
         "int64_t hi = a->ke[t] < a->Nk ? a->ke[t] : a->Nk;", "int64_t hi = a->Nk;"),
     "top-k ties to the higher column": ("return (a->j > b->j) - (a->j < b->j);",

@@ -2,12 +2,21 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl ours|reference]
 
-One step = one pass of the indexer over one batch of the chosen workload
-(default: 16 decode requests, one query token each, log-normal contexts of
-1,536-43,876 tokens, page size 64).  The K timed steps are captured in one
-CUDA graph and replayed between CUDA events on the launching stream, after W
-untimed warm-up steps; the steps rotate over enough copies of the inputs
-that their total exceeds twice the 126 MB L2, so every step reads HBM.
+One step = one pass of the indexer over one batch of a workload.  By default
+all five workloads are timed one after another and printed as ONE JSON line:
+the headline is the long-context speculative decode (16 requests, 4 query
+tokens each, log-normal contexts of 3,508-102,400 tokens, page size 64), the
+workload whose HBM roofline fraction is the decode target; the other four
+(single-request decode, 16-request decode, the 8,192-row prefill, the
+4 x 4,096-row prefill with top-512) are records under "configs", each with
+its own roofline, clocks, end-to-end and CPU-baseline figures.  `--config c`
+times one workload only.
+
+For each workload the K timed steps are captured in one CUDA graph and
+replayed between CUDA events on the launching stream, after W untimed
+warm-up steps; decode steps rotate over enough copies of the inputs that
+their total exceeds twice the 126 MB L2, and prefill steps write more than
+L2 of scores, so every step reads and writes HBM.
 
 Throughput accounting follows the vLLM PR "Separate prefill and decode
 paths for QSA indexer" (section "Microbenchmarks"), whose printed numbers
@@ -15,7 +24,8 @@ these formulas reproduce (tests/test_bench_accounting.py):
   decode bytes  = sum_b [(ctx_b // 4) * 256 + DQL * (ctx_b // 4) * 4] + B * DQL * 1024
   prefill FLOPs = 2 * 4 * 128 * sum_t visible(t)
 
-Under torchrun each rank runs its own replica of the workload (weak
+With --gpus N each of N ranks (started by torchrun, or by this script when
+no launcher set WORLD_SIZE) runs its own replica of the workload (weak
 scaling: the indexer needs no exchange between GPUs); the step time is the
 maximum over ranks and the value counts the work of all ranks.
 """
@@ -266,6 +276,34 @@ class PrefillBench:
     def throughput(self, seconds_per_step: float) -> float:
         return self.units / seconds_per_step / 1e12
 
+    def topk_bytes(self) -> int:
+        """Algorithmic bytes of the top-k step: every score read once, every
+        index written once."""
+        p = self.inp
+        return p.T * p.W * 4 + p.T * wl.TOPK_K * 4
+
+    def time_fused(self, workspace_mib: int = 64, reps: int = 10):
+        """qsa_mqa_prefill_topk through a workspace of about `workspace_mib`
+        MiB (scores of a chunk of rows stay in the 126 MB L2 between the two
+        kernels): median seconds per step over `reps`, CUDA events."""
+        if not self.topk:
+            return None
+        p = self.inp
+        ws = torch.empty(workspace_mib * 2**20 // 4, dtype=torch.float32, device=self.dev)
+        run = lambda: self.qsa.mqa_prefill_topk(self.q, self.k, self.ks, self.ke, p.W, wl.TOPK_K, ws, idx=self.idx)
+        for _ in range(3):
+            run()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, e in ev:
+            a.record()
+            run()
+            e.record()
+        torch.cuda.synchronize()
+        t = statistics.median(a.elapsed_time(e) for a, e in ev) / 1e3
+        rows = ((workspace_mib * 2**20 - 4096) // (p.W * 4)) // 64 * 64
+        return {"us_per_step": t * 1e6, "workspace_mib": workspace_mib, "rows_per_chunk": int(rows),
+                "launches_per_step": 2 * -(-p.T // rows), "tflops": self.units / t / 1e12}
+
     def e2e_setup(self):
         p = self.inp
         self.host = [t.pin_memory() for t in (p.q, p.k, p.cu_seqlens_q, p.seq_lens, p.key_offsets)]
@@ -406,13 +444,16 @@ def cpu_baseline(b, budget_s: float = 10.0) -> dict:
 
 # ------------------------------------------------------------------ main
 
+HEADLINE = 3            # the long-context spec-decode workload: the decode roofline target
+ALL_CONFIGS = [3, 1, 2, 4, 5]
+
+
 def run_reference(args, rank: int, world: int):
     """The oracle as the reference arm, timed on the host cores."""
     if rank != 0:
         return
-    dev = torch.device("cpu")
     import oracle
-    inp_bench = _HostOnly(args.config, args.kv_fp8)
+    inp_bench = _HostOnly(args.config or HEADLINE, args.kv_fp8)
     threads = oracle.default_threads()
     frac, what = inp_bench.oracle_sample()
     for _ in range(args.warmup):
@@ -473,34 +514,13 @@ class _HostOnly:
             PrefillBench.oracle_step(self, threads)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kv-fp8", action="store_true", help="decode over the fp8 E4M3 key cache")
-    ap.add_argument("--soak", type=float, default=1.5, help="seconds of load before the timed region")
-    args = ap.parse_args()
-    if args.warmup < 3:
-        ap.error("at least 3 warm-up steps")
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        run_reference(args, rank, world)
-        return
+def measure(cfg: int, args, world: int, rank: int, local: int, cpu_budget_s: float) -> dict | None:
+    """Time one workload: W eager warm-up steps, then K steps in one CUDA
+    graph between CUDA events (max over ranks); the same steps end to end
+    through the public binding; the oracle on the host cores (rank 0, N = 1).
+    Returns rank 0's record (None on the other ranks)."""
     dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=dev)
-
-    b = make_bench(args.config, dev, seed=rank, fp8=args.kv_fp8)
+    b = make_bench(cfg, dev, seed=rank, fp8=args.kv_fp8 and cfg in (1, 2, 3))
     for i in range(args.warmup):
         b.step(i)
     torch.cuda.synchronize()
@@ -508,15 +528,25 @@ def main():
     per_step, clocks = time_graph(b, args.steps, world, soak_s=args.soak, sampler=sampler)
     per_step = max_over_ranks(per_step, world)
     kernel_s = per_step
-    split = None
+    extra = {}
     if b.launches_per_step == 2:
         pre, top = time_kernel_split(b)
+        pre, top = max_over_ranks(pre, world), max_over_ranks(top, world)
         kernel_s = pre
-        split = {"prefill_us": pre * 1e6, "topk_us": top * 1e6}
+        topk_bytes = b.topk_bytes()
+        peaks = read_peaks()
+        extra["kernels"] = {
+            "prefill_us": pre * 1e6, "topk_us": top * 1e6,
+            "topk": {"bound": "hbm", "achieved": topk_bytes / top / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": topk_bytes / top / 1e9 / peaks["hbm_gbs"], "bytes_per_step": topk_bytes,
+                     "traffic": read_traffic("topk_stream_kernel", b.name)}}
+        fused = b.time_fused()
+        if fused is not None:
+            extra["fused_l2_workspace"] = fused
     e2e_s = max_over_ranks(time_e2e(b, args.steps, 3, world), world)
     from sparse_attention_block_qsa_b200 import device_error
     dev_err = device_error()
-
+    rec = None
     if rank == 0:
         peaks = read_peaks()
         value = b.throughput(per_step) * world
@@ -530,27 +560,104 @@ def main():
                     "traffic": read_traffic(b.kernel, b.name), "kernel": b.kernel,
                     "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst figure)"
                     if peaks["source"] == "measured" else "fallback"}
-        pub = None if args.kv_fp8 else PUBLISHED.get(args.config)
-        cfg = dict(b.config)
+        pub = None if args.kv_fp8 else PUBLISHED.get(cfg)
+        conf = dict(b.config)
         if pub:
-            cfg["published_reference"] = pub[2]
-        line = {"metric": METRIC, "value": value, "unit": b.unit, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": per_step * 1e3, "us_per_step": per_step * 1e6,
-                "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": (value / pub[1]) if pub and pub[0] == b.unit else None,
-                "dtype": getattr(b, "dtype", "bf16"), "data": "synthetic", "config": cfg,
-                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                "roofline": roofline,
-                "e2e": {"value": b.throughput(e2e_s) * world, "unit": b.unit, "h2d_bytes_per_step": b.h2d,
-                        "d2h_bytes_per_step": b.d2h, "ms_per_step": e2e_s * 1e3},
-                "gpu_launches": args.steps * b.launches_per_step,
-                "clocks": clocks, "device_error": dev_err}
-        if split:
-            line["kernels"] = split
+            conf["published_reference"] = pub[2]
+        rec = {"workload": b.name, "value": value, "unit": b.unit, "ms_per_step": per_step * 1e3,
+               "us_per_step": per_step * 1e6,
+               "vs_baseline": (value / pub[1]) if pub and pub[0] == b.unit else None,
+               "dtype": getattr(b, "dtype", "bf16"), "config": conf, "roofline": roofline,
+               "e2e": {"value": b.throughput(e2e_s) * world, "unit": b.unit, "h2d_bytes_per_step": b.h2d,
+                       "d2h_bytes_per_step": b.d2h, "ms_per_step": e2e_s * 1e3},
+               "gpu_launches": args.steps * b.launches_per_step, "clocks": clocks, "device_error": dev_err}
+        rec.update(extra)
         if world == 1 and not args.no_cpu_baseline:
-            cb = cpu_baseline(b)
+            cb = cpu_baseline(b, cpu_budget_s)
             cb.pop("seconds_per_step", None)
-            line["cpu_baseline"] = cb
+            rec["cpu_baseline"] = cb
+    del b
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+def relaunch(n: int) -> int:
+    """`--gpus N` without a launcher: start N replica ranks of this script
+    with torch.distributed.run on 127.0.0.1 and return its exit code."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = launch_command(sys.argv[1:], n, port)
+    return subprocess.run(cmd).returncode
+
+
+def launch_command(argv: list[str], n: int, port: int, script: str | None = None) -> list[str]:
+    """torchrun command line that starts `script` (this file) on n ranks of one node."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", script or os.path.abspath(__file__), *argv]
+
+
+def check_world(gpus: int, env) -> tuple[int, int, int]:
+    """(world, rank, local rank) of this process; the world size must be the
+    requested GPU count."""
+    world = int(env.get("WORLD_SIZE", "1"))
+    if world != gpus:
+        raise SystemExit(f"bench.py: --gpus {gpus} but WORLD_SIZE={world}; launch one rank per GPU "
+                         f"(or run without a launcher and let --gpus start the ranks)")
+    return world, int(env.get("RANK", "0")), int(env.get("LOCAL_RANK", "0"))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=None, choices=[1, 2, 3, 4, 5],
+                    help="one workload only (default: all five, the long-context spec-decode one as the headline)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-fp8", action="store_true", help="decode over the fp8 E4M3 key cache")
+    ap.add_argument("--soak", type=float, default=1.5, help="seconds of load before each timed region")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch(args.gpus))
+    world, rank, local = check_world(args.gpus, os.environ)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    configs = [args.config] if args.config else ALL_CONFIGS
+    records = {}
+    for i, cfg in enumerate(configs):
+        records[cfg] = measure(cfg, args, world, rank, local, cpu_budget_s=10.0 if i == 0 else 5.0)
+
+    if rank == 0:
+        head = records[configs[0]]
+        line = {"metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+                "us_per_step": head["us_per_step"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": head["vs_baseline"], "dtype": head["dtype"], "data": "synthetic",
+                "config": head["config"],
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "roofline": head["roofline"], "e2e": head["e2e"],
+                "gpu_launches": sum(r["gpu_launches"] for r in records.values()),
+                "clocks": head["clocks"], "device_error": max(r["device_error"] for r in records.values())}
+        for key in ("kernels", "fused_l2_workspace", "cpu_baseline"):
+            if key in head:
+                line[key] = head[key]
+        if len(configs) > 1:
+            line["configs"] = {records[c]["workload"]: records[c] for c in configs[1:]}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

@@ -26,8 +26,8 @@
  *    The library allocates nothing, never synchronises the stream and never
  *    reads device memory from the host; every call is asynchronous on
  *    `stream` (a cudaStream_t; NULL means the legacy default stream).
- *  - bf16 tensors are passed as raw pointers with strides in ELEMENTS; the
- *    feature (last) stride is always 1.
+ *  - bf16 / fp16 tensors are passed as raw pointers with strides in ELEMENTS;
+ *    the feature (last) stride is always 1.
  *  - Host-side validation runs before any launch.  On a non-OK status nothing
  *    was launched and qsa_last_error_detail() describes the problem.
  *  - Kernels never trap.  A device-side wait that runs out of time sets a bit
@@ -95,7 +95,10 @@ qsa_status_t qsa_selftest_bounded_wait(uint64_t timeout_ns, int32_t arrive, void
  *   k_cache    bf16 [num_pages, page_size, 1, 128]; row r of page p at
  *              k_cache + p*k_page_stride + r*k_row_stride.  16-byte aligned,
  *              both strides multiples of 8, k_row_stride >= 128.
- *   page_size  8, 16, 32 or 64.
+ *   page_size  8 .. 1024 rows per page.  The QSA docs list 8, 16, 32 and 64
+ *              as the native sizes; the vLLM PR measures at 196, its
+ *              production size.  Sizes that are not powers of two take a
+ *              per-key page lookup (integer multiply-shift division).
  *   page_table int32 [B, max_pages], row stride pt_stride (>= max_pages).
  *              Key n of request b lives in page page_table[b, n / page_size]
  *              at row n % page_size.  Entries may be -1; an entry that is
@@ -111,15 +114,25 @@ qsa_status_t qsa_selftest_bounded_wait(uint64_t timeout_ns, int32_t arrive, void
  *              every n < W (columns past the visible keys are filled with
  *              -inf).  W >= max visible is the caller's choice; keys at
  *              n >= W are not scored.  out must not overlap any input.
- *              Limit: min(B, 8192) * ceil(W / 8) must stay below 2^32 (the
- *              kernel counts 8-key tiles in 32 bits; reaching it takes an
- *              output of more than 128 GB); it is not checked.
+ *              Requests are launched in groups of at most
+ *              min(8192, floor((2^32 - 1) / ceil(W / 8))) so that the
+ *              kernel's 32-bit count of 8-key tiles cannot overflow.
  */
 qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
                             const void* k_cache, int64_t num_pages, int32_t page_size, int64_t k_page_stride,
                             int64_t k_row_stride, const int32_t* page_table, int64_t pt_stride,
                             int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t Q, float scale,
                             float* out, int64_t out_stride_b, int64_t out_stride_t, int32_t W, void* stream);
+
+/* qsa_mqa_decode_f16 - qsa_mqa_decode with fp16 q and k_cache (QSA docs,
+ * MATE, section "MQA score": queries and keys are BF16 or FP16).  The
+ * products accumulate in fp32 as for bf16; arguments, layout and errors as
+ * qsa_mqa_decode. */
+qsa_status_t qsa_mqa_decode_f16(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
+                                const void* k_cache, int64_t num_pages, int32_t page_size, int64_t k_page_stride,
+                                int64_t k_row_stride, const int32_t* page_table, int64_t pt_stride,
+                                int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t Q, float scale,
+                                float* out, int64_t out_stride_b, int64_t out_stride_t, int32_t W, void* stream);
 
 /*
  * qsa_mqa_decode_fp8 - qsa_mqa_decode over an fp8 E4M3 compressed key cache.
@@ -164,11 +177,21 @@ qsa_status_t qsa_mqa_decode_fp8(const void* q, int64_t q_stride_b, int64_t q_str
  *   out      fp32 [T, W], row stride out_stride (>= W when T > 1):
  *            out[t, j] = score(t, ks[t] + j) if that key is in the row's
  *            interval, else -inf, for every j < W.  Must not overlap inputs.
- *   T        rows, 0 <= T <= 16,777,216.
+ *   T        rows, 0 <= T <= 2^31 - 1 (larger T returns
+ *            QSA_ERR_UNSUPPORTED); the rows are launched in groups of at
+ *            most 131,072.
  */
 qsa_status_t qsa_mqa_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
                              int64_t k_stride, int64_t Nk, const int32_t* ks, const int32_t* ke, int64_t T,
                              float scale, float* out, int64_t out_stride, int32_t W, void* stream);
+
+/* qsa_mqa_prefill_f16 - qsa_mqa_prefill with fp16 q and k (QSA docs, MATE,
+ * section "MQA score": queries and keys are BF16 or FP16).  The products
+ * accumulate in fp32 as for bf16; arguments, layout and errors as
+ * qsa_mqa_prefill. */
+qsa_status_t qsa_mqa_prefill_f16(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
+                                 int64_t k_stride, int64_t Nk, const int32_t* ks, const int32_t* ke, int64_t T,
+                                 float scale, float* out, int64_t out_stride, int32_t W, void* stream);
 
 /*
  * qsa_prefill_intervals - per-row key intervals of a packed prefill batch,

@@ -26,6 +26,10 @@ SIGNATURES = {
     "qsa_selftest_bounded_wait": (C.c_int, [C.c_uint64, _i32, _vp]),
     "qsa_mqa_decode": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _i64, _i32, _i64, _i64, _vp, _i64, _i32,
                                  _vp, _i32, _i32, _f32, _vp, _i64, _i64, _i32, _vp]),
+    "qsa_mqa_decode_f16": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _i64, _i32, _i64, _i64, _vp, _i64, _i32,
+                                     _vp, _i32, _i32, _f32, _vp, _i64, _i64, _i32, _vp]),
+    "qsa_mqa_prefill_f16": (C.c_int, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f32, _vp, _i64,
+                                      _i32, _vp]),
     "qsa_mqa_decode_fp8": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _f32, _i64, _i32, _i64, _i64, _vp, _i64,
                                      _i32, _vp, _i32, _i32, _f32, _vp, _i64, _i64, _i32, _vp]),
     "qsa_mqa_prefill": (C.c_int, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f32, _vp, _i64,
@@ -105,8 +109,8 @@ def selftest_bounded_wait(timeout_ns: int, arrive: bool, stream=None) -> None:
                                                                        _stream(stream)))
 
 
-def _decode_checks(q, k_cache, page_table, seq_lens, W, out):
-    _need(q, "q", torch.bfloat16, 4)
+def _decode_checks(q, k_cache, page_table, seq_lens, W, out, q_dtype=torch.bfloat16):
+    _need(q, "q", q_dtype, 4)
     _need(page_table, "page_table", torch.int32, 2)
     _need(seq_lens, "seq_lens", torch.int32, 1)
     B, Q = q.shape[0], q.shape[1]
@@ -126,12 +130,14 @@ def _decode_checks(q, k_cache, page_table, seq_lens, W, out):
 
 def mqa_decode(q: torch.Tensor, k_cache: torch.Tensor, page_table: torch.Tensor, seq_lens: torch.Tensor,
                W: int, scale: float = SCALE, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Decode / spec-decode scores: q bf16 [B, Q, 4, 128], k_cache bf16
-    [pages, page_size, 1, 128], page_table int32 [B, max_pages], seq_lens int32
-    [B] (tokens) -> out fp32 [B, Q, W]."""
-    _need(k_cache, "k_cache", torch.bfloat16, 4)
-    B, Q, out = _decode_checks(q, k_cache, page_table, seq_lens, W, out)
-    _check("qsa_mqa_decode", lib().qsa_mqa_decode(
+    """Decode / spec-decode scores: q [B, Q, 4, 128] and k_cache [pages,
+    page_size, 1, 128] both bf16 or both fp16, page_table int32 [B,
+    max_pages], seq_lens int32 [B] (tokens) -> out fp32 [B, Q, W]."""
+    dt = q.dtype if isinstance(q, torch.Tensor) and q.dtype == torch.float16 else torch.bfloat16
+    _need(k_cache, "k_cache", dt, 4)
+    B, Q, out = _decode_checks(q, k_cache, page_table, seq_lens, W, out, dt)
+    name = "qsa_mqa_decode_f16" if dt == torch.float16 else "qsa_mqa_decode"
+    _check(name, getattr(lib(), name)(
         _ptr(q), q.stride(0), q.stride(1), q.stride(2),
         _ptr(k_cache), k_cache.shape[0], k_cache.shape[1], k_cache.stride(0), k_cache.stride(1),
         _ptr(page_table), page_table.stride(0), page_table.shape[1], _ptr(seq_lens), B, Q, scale,
@@ -157,9 +163,9 @@ def mqa_decode_fp8(q: torch.Tensor, k_cache: torch.Tensor, k_scale: float, page_
     return out
 
 
-def _prefill_checks(q, k, ks, ke):
-    _need(q, "q", torch.bfloat16, 3)
-    _need(k, "k", torch.bfloat16, 2)
+def _prefill_checks(q, k, ks, ke, dt=torch.bfloat16):
+    _need(q, "q", dt, 3)
+    _need(k, "k", dt, 2)
     _need(ks, "ks", torch.int32, 1)
     _need(ke, "ke", torch.int32, 1)
     if q.shape[1:] != (4, 128) or q.stride(2) != 1:
@@ -172,16 +178,18 @@ def _prefill_checks(q, k, ks, ke):
 
 def mqa_prefill(q: torch.Tensor, k: torch.Tensor, ks: torch.Tensor, ke: torch.Tensor, W: int,
                 scale: float = SCALE, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Prefill scores: q bf16 [T, 4, 128], k bf16 [Nk, 128], ks/ke int32 [T]
-    -> out fp32 [T, W] with out[t, j] the score of key ks[t] + j."""
-    _prefill_checks(q, k, ks, ke)
+    """Prefill scores: q [T, 4, 128] and k [Nk, 128] both bf16 or both fp16,
+    ks/ke int32 [T] -> out fp32 [T, W] with out[t, j] the score of key ks[t] + j."""
+    dt = q.dtype if isinstance(q, torch.Tensor) and q.dtype == torch.float16 else torch.bfloat16
+    _prefill_checks(q, k, ks, ke, dt)
     T = q.shape[0]
     if out is None:
         out = torch.empty((T, W), dtype=torch.float32, device=q.device)
     _need(out, "out", torch.float32, 2)
     if out.shape[0] != T or out.stride(1) != 1:
         raise ValueError("out must be [T, W] with unit column stride")
-    _check("qsa_mqa_prefill", lib().qsa_mqa_prefill(
+    name = "qsa_mqa_prefill_f16" if dt == torch.float16 else "qsa_mqa_prefill"
+    _check(name, getattr(lib(), name)(
         _ptr(q), q.stride(0), q.stride(1), _ptr(k), k.stride(0), k.shape[0], _ptr(ks), _ptr(ke), T, scale,
         _ptr(out), out.stride(0), out.shape[1], _stream(stream)))
     return out

@@ -71,7 +71,10 @@ struct Params {
   const int32_t* seq_lens;
   int32_t B;
   int32_t Q;
-  int32_t log2_ps;
+  int32_t log2_ps;          // page size 2^log2_ps (power-of-two instance)
+  uint32_t ps;              // page size (any-size instance): key n is in page n / ps, row n % ps
+  uint32_t ps_magic;        // n / ps == (n * ps_magic) >> ps_shift for every key index n < 2^31
+  int32_t ps_shift;
   float scale;              // fp8 cache: scale * k_scale
   float* out;
   int64_t out_sb;
@@ -80,6 +83,10 @@ struct Params {
 };
 
 constexpr size_t SMEM_BYTES = sizeof(int32_t) * (MAX_B + 1);
+
+// Element format of q and the key cache: bf16 q and keys, fp16 q and keys,
+// or bf16 q over an fp8 E4M3 cache.
+enum class Fmt { BF16, F16, E4M3 };
 
 // Keys of a request that can be visible in a column < W: the last query
 // token sees seq_len / 4 of them.
@@ -157,7 +164,7 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint
 // Query fragments of request b: A = 16 rows (row = head * 4 + token) x 128.
 // fp8 cache: fp16 fragments of the scaled rows, and in up0 / up1 the factors
 // that undo the scaling of rows g and g + 8.
-template <bool FP8>
+template <Fmt F>
 __device__ __forceinline__ void load_queries(const Params& p, int b, int lane, uint32_t (&a)[8][4], float& up0,
                                              float& up1) {
   const int g = lane >> 2, c = lane & 3;
@@ -174,7 +181,7 @@ __device__ __forceinline__ void load_queries(const Params& p, int b, int lane, u
     w0[4 * i] = x.x; w0[4 * i + 1] = x.y; w0[4 * i + 2] = x.z; w0[4 * i + 3] = x.w;
     w1[4 * i] = y.x; w1[4 * i + 1] = y.y; w1[4 * i + 2] = y.z; w1[4 * i + 3] = y.w;
   }
-  if constexpr (FP8) {
+  if constexpr (F == Fmt::E4M3) {
     uint32_t m0 = 0, m1 = 0;  // largest magnitude bits of rows g and g + 8 (this lane's 32 features)
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -204,8 +211,21 @@ __device__ __forceinline__ void load_queries(const Params& p, int b, int lane, u
   }
 }
 
-template <bool FP8>
+// Logical page of key n and its row in that page.
+template <bool GEN>
+__device__ __forceinline__ void page_of(const Params& p, int n, int& lp, int& row) {
+  if constexpr (GEN) {
+    lp = (int)(((uint64_t)(uint32_t)n * p.ps_magic) >> p.ps_shift);
+    row = n - lp * (int)p.ps;
+  } else {
+    lp = n >> p.log2_ps;
+    row = n & ((1 << p.log2_ps) - 1);
+  }
+}
+
+template <Fmt F, bool GEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) {
+  constexpr bool FP8 = F == Fmt::E4M3;
   constexpr int NB = FP8 ? 2 * BATCH : BATCH;  // tiles in flight per warp
   extern __shared__ int32_t prefix[];  // prefix[b]: tiles before request b
   __shared__ uint32_t red[WARPS];
@@ -364,21 +384,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   const int g = lane >> 2, c = lane & 3;
   const int t = g & 3;                  // token of this lane's rows
   const int key = 2 * c + (lane >> 4);  // key of a tile this lane stores
-  const int ps_mask = (1 << p.log2_ps) - 1;
   uint32_t qa[8][4];
   float up0 = 1.f, up1 = 1.f;
-  load_queries<FP8>(p, b, lane, qa, up0, up1);
+  load_queries<F>(p, b, lane, qa, up0, up1);
   int L = __ldg(p.seq_lens + b);
   int nt_b = (int)(pfx(b + 1) - pfx(b));
-  // Page of tile j0 + lane of the current request, read 32 tiles ahead so
-  // that no page-table load sits between two batches of key loads.
+  // Page entries of the current request, read 32 tiles ahead so that no
+  // page-table load sits between two batches of key loads.  Power-of-two
+  // pages: lane l holds the page of tile j0 + l (a tile never straddles a
+  // page).  Any page size >= 8: lane l holds logical page lp0 + l, where lp0
+  // is the page of tile j0's first key; 32 pages of >= 8 rows cover the 32
+  // tiles j0 .. j0 + 31.
   int j0 = j;
   int entry = -1;
+  int lp0 = 0;
   // The raw entry stays a pending load until a batch reads it; the range
   // check happens there.
   auto fetch_entries = [&]() {
-    const int tile = min(j0 + lane, nt_b - 1);
-    const int logical = min((tile * TILE) >> p.log2_ps, p.max_pages - 1);
+    int logical;
+    if constexpr (GEN) {
+      int row0;
+      page_of<true>(p, j0 * TILE, lp0, row0);
+      logical = min(lp0 + lane, p.max_pages - 1);
+    } else {
+      const int tile = min(j0 + lane, nt_b - 1);
+      logical = min((tile * TILE) >> p.log2_ps, p.max_pages - 1);
+    }
     entry = p.max_pages > 0 ? __ldg(p.page_table + (int64_t)b * p.pt_stride + logical) : -1;
   };
   fetch_entries();
@@ -387,16 +418,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
     const int cnt = (int)min((uint32_t)min(min(NB, nt_b - j), 32 - (j - j0)), left);
     uint4 kv[FP8 ? 1 : NB][4];   // bf16: chunk i = 16 bytes
     uint2 kv8[FP8 ? NB : 1][4];  // fp8: chunk i = 8 bytes
-    uint32_t valid = 0;  // bit u: tile u has a page
+    uint32_t valid = 0;  // bit u: the page of key g of tile u (this lane's loads) is valid
 #pragma unroll
     for (int u = 0; u < NB; ++u) {
-      const int ent = __shfl_sync(0xffffffffu, entry, (j - j0 + u) & 31);
-      // tiles past the request's pages (logical page >= max_pages) and
+      // keys past the request's pages (logical page >= max_pages) and
       // entries outside the pool are invalid
-      const bool in_table = (((j + u) * TILE) >> p.log2_ps) < p.max_pages;
-      const bool ok = in_table && ent >= 0 && (int64_t)ent < p.num_pages;
+      int lp, row;
+      page_of<GEN>(p, (j + u) * TILE + g, lp, row);
+      const int src = GEN ? (lp - lp0) & 31 : (j - j0 + u) & 31;
+      const int ent = __shfl_sync(0xffffffffu, entry, src);
+      const bool ok = lp < p.max_pages && ent >= 0 && (int64_t)ent < p.num_pages;
       valid |= ok ? 1u << u : 0u;
-      const int row = ((j + u) * TILE + g) & ps_mask;
       const int64_t off = (int64_t)ent * p.k_page_stride + (int64_t)row * p.k_row_stride;
       if constexpr (FP8) {
         if (u < cnt && ok) {
@@ -416,6 +448,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
         }
       }
     }
+    // validity of the key this lane stores (key 2c + lane / 16), held by the
+    // lanes that loaded it (4 * key .. 4 * key + 3); uniform over a tile
+    // when pages hold whole tiles
+    const uint32_t vst = GEN ? __shfl_sync(0xffffffffu, valid, key << 2) : valid;
     const int vis = t < p.Q ? visible_of(L, p.Q, t) : 0;
     const int jb = j;
     j += cnt;
@@ -450,6 +486,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
             // words 2s, 2s + 1 = bytes 0-3 (s even) or 4-7 (s odd) of chunk s / 2
             const uint32_t four = (s & 1) ? kv8[u0 + v][s >> 1].y : kv8[u0 + v][s >> 1].x;
             mma_f16_16816(d[v], qa[s], e4m3x2_to_f16x2(four), e4m3x2_to_f16x2(four >> 16));
+          } else if constexpr (F == Fmt::F16) {
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[u0 + v]);
+            mma_f16_16816(d[v], qa[s], w[2 * s], w[2 * s + 1]);
           } else {
             const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[u0 + v]);
             mma_bf16_16816(d[v], qa[s], w[2 * s], w[2 * s + 1]);
@@ -474,7 +513,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
           const int n = (jb + u) * TILE + key;
           if (t < p.Q && n < p.W) {
             const float sc = p.scale * ((lane >> 4) ? s1 : s0);
-            p.out[(int64_t)ob * p.out_sb + (int64_t)t * p.out_st + n] = ((valid >> u) & 1u) && n < vis ? sc : -INFINITY;
+            p.out[(int64_t)ob * p.out_sb + (int64_t)t * p.out_st + n] = ((vst >> u) & 1u) && n < vis ? sc : -INFINITY;
           }
         }
       }
@@ -482,7 +521,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
     if (ob != b) {
       ob = b;
       L = __ldg(p.seq_lens + b);
-      load_queries<FP8>(p, b, lane, qa, up0, up1);
+      load_queries<F>(p, b, lane, qa, up0, up1);
     }
   }
   fill_tail();

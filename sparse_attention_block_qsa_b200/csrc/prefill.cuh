@@ -50,6 +50,7 @@ constexpr int STAGING_BYTES = EPI_WARPS * WARP_STAGE_BYTES;
 constexpr int MAX_TT = 2048;         // token tiles per launch
 constexpr int64_t MAX_ROWS_PER_LAUNCH = (int64_t)MAX_TT * BT;
 constexpr uint32_t IDESC = umma_idesc_bf16_f32(BM, BN);
+constexpr uint32_t IDESC_F16 = umma_idesc_f16_f32(BM, BN);
 
 struct Params {
   const int32_t* ks;   // rows of this launch
@@ -154,6 +155,7 @@ struct Walk {
   __device__ __forceinline__ int kt() const { return kt0 + i; }
 };
 
+template <bool F16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_out, const Params p) {
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         umma_bf16_k128<KHALF_BYTES / 16, QHALF_BYTES / 16>(tmem_base + a * BN,
-                                                           kdesc0 + (uint64_t)(s * (K_STAGE_BYTES / 16)), qdesc, IDESC);
+                                                           kdesc0 + (uint64_t)(s * (K_STAGE_BYTES / 16)), qdesc, F16 ? IDESC_F16 : IDESC);
         umma_commit(&S.empty[s]);
         umma_commit(&S.acc_full[a]);
         last = it;

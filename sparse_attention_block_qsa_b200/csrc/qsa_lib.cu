@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -68,11 +69,12 @@ EncodeTiledFn encode_fn() {
 }
 
 qsa_status_t encode_bf16_map(CUtensorMap* map, int rank, void* base, const cuuint64_t* dims,
-                             const cuuint64_t* strides_bytes, const cuuint32_t* box, const char* what) {
+                             const cuuint64_t* strides_bytes, const cuuint32_t* box, const char* what,
+                             bool f16 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides_bytes, box, estr,
+  CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides_bytes, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(QSA_ERR_ALIGNMENT, "tensor map for %s rejected by the driver (CUresult %d)", what, (int)r);
@@ -126,9 +128,14 @@ qsa_status_t device_info(int* sms) {
       const void* fn;
       size_t bytes;
     } kernels[] = {
-        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<false>), qsa::decode::SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<true>), qsa::decode::SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel), qsa::prefill::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::BF16, false>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::BF16, true>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::F16, false>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::F16, true>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::E4M3, false>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::E4M3, true>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel<false>), qsa::prefill::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel<true>), qsa::prefill::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_rows_kernel), qsa::topk::ROWS_SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_stream_kernel), qsa::topk::STREAM_SMEM_BYTES},
     };
@@ -183,6 +190,7 @@ struct PrefillArgs {
   float* out;
   int64_t out_stride;
   int32_t W;
+  bool f16 = false;  // q and k hold fp16 instead of bf16
 };
 
 qsa_status_t validate_prefill(const PrefillArgs& a) {
@@ -225,14 +233,14 @@ qsa_status_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     cuuint64_t dims[3] = {128, 4, (cuuint64_t)a.T};
     cuuint64_t strides[2] = {(cuuint64_t)a.q_stride_h * 2, (cuuint64_t)st_t * 2};
     cuuint32_t box[3] = {64, 4, (cuuint32_t)qsa::prefill::BT};
-    st = encode_bf16_map(&tm_q, 3, const_cast<void*>(a.q), dims, strides, box, "q");
+    st = encode_bf16_map(&tm_q, 3, const_cast<void*>(a.q), dims, strides, box, "q", a.f16);
     if (st != QSA_OK) return st;
   }
   if (a.Nk > 0) {
     cuuint64_t dims[2] = {128, (cuuint64_t)a.Nk};
     cuuint64_t strides[1] = {(cuuint64_t)(a.Nk > 1 ? a.k_stride : 128) * 2};
     cuuint32_t box[2] = {64, (cuuint32_t)qsa::prefill::BM};
-    st = encode_bf16_map(&tm_k, 2, const_cast<void*>(a.k), dims, strides, box, "k");
+    st = encode_bf16_map(&tm_k, 2, const_cast<void*>(a.k), dims, strides, box, "k", a.f16);
     if (st != QSA_OK) return st;
   }
   for (int64_t r0 = 0; r0 < a.T; r0 += qsa::prefill::MAX_ROWS_PER_LAUNCH) {
@@ -249,8 +257,12 @@ qsa_status_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     CUtensorMap tm_out;
     memset(&tm_out, 0, sizeof tm_out);
     p.store_map = encode_f32_store_map(&tm_out, p.out, a.W, p.T, a.out_stride) ? 1 : 0;
-    qsa::prefill::prefill_kernel<<<sms, qsa::prefill::NUM_THREADS, qsa::prefill::SMEM_BYTES, stream>>>(
-        tm_q, tm_k, tm_out, p);
+    if (a.f16)
+      qsa::prefill::prefill_kernel<true><<<sms, qsa::prefill::NUM_THREADS, qsa::prefill::SMEM_BYTES, stream>>>(
+          tm_q, tm_k, tm_out, p);
+    else
+      qsa::prefill::prefill_kernel<false><<<sms, qsa::prefill::NUM_THREADS, qsa::prefill::SMEM_BYTES, stream>>>(
+          tm_q, tm_k, tm_out, p);
     st = launch_status("prefill kernel");
     if (st != QSA_OK) return st;
   }
@@ -288,6 +300,11 @@ qsa_status_t validate_topk(const TopkArgs& a) {
   return QSA_OK;
 }
 
+// Bytes at the end of a fused prefill + top-k workspace that carry the top-k
+// kernel's per-CTA threshold predictions from one chunk to the next.
+constexpr size_t kPredBytes = 4096;
+constexpr int64_t kPredFloats = kPredBytes / sizeof(float);
+
 qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream, float* pred_state = nullptr) {
   int sms = 0;
   qsa_status_t st = device_info(&sms);
@@ -303,13 +320,15 @@ qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream, float* pred_sta
   p.vec4 = aligned(a.scores, 16) && (p.stride % 4 == 0);
   p.rows = a.rows;
   p.pred_state = pred_state;
+  // the predictions carried between chunks hold one float per CTA
+  const int64_t max_grid = pred_state ? kPredFloats : INT32_MAX;
   if (p.vec4 && a.W % 4 == 0) {
     // rows start on 16-byte boundaries: stream them with bulk copies
-    const int64_t grid = std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::STREAM_CTAS_PER_SM);
+    const int64_t grid = std::min<int64_t>(std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::STREAM_CTAS_PER_SM), max_grid);
     qsa::topk::topk_stream_kernel<<<(unsigned)grid, qsa::topk::STREAM_THREADS, qsa::topk::STREAM_SMEM_BYTES,
                                     stream>>>(p);
   } else {
-    const int64_t grid = std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::ROWS_CTAS_PER_SM);
+    const int64_t grid = std::min<int64_t>(std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::ROWS_CTAS_PER_SM), max_grid);
     qsa::topk::topk_rows_kernel<<<(unsigned)grid, qsa::topk::THREADS, qsa::topk::ROWS_SMEM_BYTES, stream>>>(p);
   }
   return launch_status("top-k kernel");
@@ -374,18 +393,27 @@ qsa_status_t qsa_selftest_bounded_wait(uint64_t timeout_ns, int32_t arrive, void
   return launch_status("self-test kernel");
 }
 
-// Both cache formats: fp8 selects E4M3 keys (1 byte per element, strides
-// multiples of 16) scaled by k_scale; otherwise bf16 keys and k_scale == 1.
+// Every format: E4M3 keys take 1 byte per element (strides multiples of 16)
+// and are scaled by k_scale; bf16 and fp16 keys take 2 (k_scale == 1).
+extern "C++" {
+template <qsa::decode::Fmt F, bool GEN>
+static void launch_decode(int sms, const qsa::decode::Params& p, cudaStream_t stream) {
+  qsa::decode::decode_kernel<F, GEN><<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES, stream>>>(p);
+}
+}
+
 static qsa_status_t decode_common(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
-                                  const void* k_cache, bool fp8, float k_scale, int64_t num_pages, int32_t page_size,
+                                  const void* k_cache, qsa::decode::Fmt fmt, float k_scale, int64_t num_pages,
+                                  int32_t page_size,
                                   int64_t k_page_stride, int64_t k_row_stride, const int32_t* page_table,
                                   int64_t pt_stride, int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t Q,
                                   float scale, float* out, int64_t out_stride_b, int64_t out_stride_t, int32_t W,
                                   void* stream) {
   if (B < 0 || W < 0) return fail(QSA_ERR_INVALID_ARG, "B and W must be non-negative");
   if (Q < 1 || Q > 4) return fail(QSA_ERR_UNSUPPORTED, "Q = %d query tokens per request; 1..4 supported", Q);
-  if (page_size != 8 && page_size != 16 && page_size != 32 && page_size != 64)
-    return fail(QSA_ERR_UNSUPPORTED, "page_size = %d; supported page sizes are 8, 16, 32 and 64", page_size);
+  if (page_size < 8 || page_size > 1024)
+    return fail(QSA_ERR_UNSUPPORTED, "page_size = %d; supported page sizes are 8 .. 1024", page_size);
+  const bool fp8 = fmt == qsa::decode::Fmt::E4M3;
   if (!std::isfinite(scale)) return fail(QSA_ERR_INVALID_ARG, "scale must be finite");
   if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(scale * k_scale)))
     return fail(QSA_ERR_INVALID_ARG, "k_scale must be finite and positive, and scale * k_scale finite");
@@ -442,24 +470,39 @@ static qsa_status_t decode_common(const void* q, int64_t q_stride_b, int64_t q_s
   p.pt_stride = pt_stride;
   p.max_pages = max_pages;
   p.Q = Q;
-  p.log2_ps = page_size == 8 ? 3 : page_size == 16 ? 4 : page_size == 32 ? 5 : 6;
+  const bool pow2 = (page_size & (page_size - 1)) == 0;
+  int log2_ps = 0;
+  while ((1 << (log2_ps + 1)) <= page_size) ++log2_ps;
+  p.log2_ps = log2_ps;
+  // Key n lies in logical page n / ps = (n * m) >> s for 0 <= n < 2^30, with
+  // s = 31 + floor(log2 ps) and m = ceil(2^s / ps) < 2^32 (ps >= 8).  Write
+  // m * ps = 2^s + e with 0 <= e < ps: then n * m / 2^s = n / ps +
+  // n * e / (ps * 2^s), and n * e < 2^30 * 2^(floor(log2 ps) + 1) = 2^s, so the
+  // extra term stays below 1 / ps and never lifts the floor past n / ps.
+  // (A request holds fewer than 2^29 keys: seq_len is an int32 of tokens.)
+  p.ps = (uint32_t)page_size;
+  p.ps_shift = 31 + log2_ps;
+  p.ps_magic = (uint32_t)(((1ull << p.ps_shift) + (uint64_t)page_size - 1) / (uint64_t)page_size);
   p.scale = fp8 ? scale * k_scale : scale;
   p.out_sb = out_stride_b;
   p.out_st = out_stride_t;
   p.W = W;
-  // requests are independent: launch them in groups that fit the kernel's prefix table
-  for (int32_t b0 = 0; b0 < B; b0 += qsa::decode::MAX_B) {
-    p.B = std::min(B - b0, qsa::decode::MAX_B);
+  // Requests are independent: launch them in groups that fit the kernel's
+  // prefix table and whose 8-key tile count, at most ceil(W / 8) per request,
+  // fits the kernel's 32-bit tile indices.
+  const int64_t tiles_per_req = ((int64_t)W + qsa::decode::TILE - 1) / qsa::decode::TILE;
+  const int32_t group = (int32_t)std::min<int64_t>(qsa::decode::MAX_B, (int64_t)UINT32_MAX / tiles_per_req);
+  for (int32_t b0 = 0; b0 < B; b0 += group) {
+    p.B = std::min(B - b0, group);
     p.q = static_cast<const uint16_t*>(q) + (int64_t)b0 * p.q_sb;
     p.page_table = max_pages > 0 ? page_table + (int64_t)b0 * pt_stride : page_table;
     p.seq_lens = seq_lens + b0;
     p.out = out + (int64_t)b0 * out_stride_b;
-    if (fp8)
-      qsa::decode::decode_kernel<true><<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES,
-                                         static_cast<cudaStream_t>(stream)>>>(p);
-    else
-      qsa::decode::decode_kernel<false><<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES,
-                                          static_cast<cudaStream_t>(stream)>>>(p);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    using qsa::decode::Fmt;
+    if (fmt == Fmt::E4M3) pow2 ? launch_decode<Fmt::E4M3, false>(sms, p, s) : launch_decode<Fmt::E4M3, true>(sms, p, s);
+    else if (fmt == Fmt::F16) pow2 ? launch_decode<Fmt::F16, false>(sms, p, s) : launch_decode<Fmt::F16, true>(sms, p, s);
+    else pow2 ? launch_decode<Fmt::BF16, false>(sms, p, s) : launch_decode<Fmt::BF16, true>(sms, p, s);
     st = launch_status("decode kernel");
     if (st != QSA_OK) return st;
   }
@@ -471,9 +514,19 @@ qsa_status_t qsa_mqa_decode(const void* q, int64_t q_stride_b, int64_t q_stride_
                             int64_t k_row_stride, const int32_t* page_table, int64_t pt_stride, int32_t max_pages,
                             const int32_t* seq_lens, int32_t B, int32_t Q, float scale, float* out,
                             int64_t out_stride_b, int64_t out_stride_t, int32_t W, void* stream) {
-  return decode_common(q, q_stride_b, q_stride_t, q_stride_h, k_cache, false, 1.f, num_pages, page_size,
-                       k_page_stride, k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale, out,
-                       out_stride_b, out_stride_t, W, stream);
+  return decode_common(q, q_stride_b, q_stride_t, q_stride_h, k_cache, qsa::decode::Fmt::BF16, 1.f, num_pages,
+                       page_size, k_page_stride, k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale,
+                       out, out_stride_b, out_stride_t, W, stream);
+}
+
+qsa_status_t qsa_mqa_decode_f16(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
+                                const void* k_cache, int64_t num_pages, int32_t page_size, int64_t k_page_stride,
+                                int64_t k_row_stride, const int32_t* page_table, int64_t pt_stride, int32_t max_pages,
+                                const int32_t* seq_lens, int32_t B, int32_t Q, float scale, float* out,
+                                int64_t out_stride_b, int64_t out_stride_t, int32_t W, void* stream) {
+  return decode_common(q, q_stride_b, q_stride_t, q_stride_h, k_cache, qsa::decode::Fmt::F16, 1.f, num_pages,
+                       page_size, k_page_stride, k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale,
+                       out, out_stride_b, out_stride_t, W, stream);
 }
 
 qsa_status_t qsa_mqa_decode_fp8(const void* q, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
@@ -482,15 +535,25 @@ qsa_status_t qsa_mqa_decode_fp8(const void* q, int64_t q_stride_b, int64_t q_str
                                 int64_t pt_stride, int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t Q,
                                 float scale, float* out, int64_t out_stride_b, int64_t out_stride_t, int32_t W,
                                 void* stream) {
-  return decode_common(q, q_stride_b, q_stride_t, q_stride_h, k_cache, true, k_scale, num_pages, page_size,
-                       k_page_stride, k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale, out,
-                       out_stride_b, out_stride_t, W, stream);
+  return decode_common(q, q_stride_b, q_stride_t, q_stride_h, k_cache, qsa::decode::Fmt::E4M3, k_scale, num_pages,
+                       page_size, k_page_stride, k_row_stride, page_table, pt_stride, max_pages, seq_lens, B, Q, scale,
+                       out, out_stride_b, out_stride_t, W, stream);
 }
 
 qsa_status_t qsa_mqa_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k, int64_t k_stride,
                              int64_t Nk, const int32_t* ks, const int32_t* ke, int64_t T, float scale, float* out,
                              int64_t out_stride, int32_t W, void* stream) {
   PrefillArgs a{q, q_stride_t, q_stride_h, k, k_stride, Nk, ks, ke, T, scale, out, out_stride, W};
+  qsa_status_t st = validate_prefill(a);
+  if (st != QSA_OK) return st;
+  if (T == 0 || W == 0) return ok();
+  return launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+qsa_status_t qsa_mqa_prefill_f16(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
+                                 int64_t k_stride, int64_t Nk, const int32_t* ks, const int32_t* ke, int64_t T,
+                                 float scale, float* out, int64_t out_stride, int32_t W, void* stream) {
+  PrefillArgs a{q, q_stride_t, q_stride_h, k, k_stride, Nk, ks, ke, T, scale, out, out_stride, W, true};
   qsa_status_t st = validate_prefill(a);
   if (st != QSA_OK) return st;
   if (T == 0 || W == 0) return ok();
@@ -528,10 +591,10 @@ qsa_status_t qsa_mqa_prefill_topk_noalloc(const void* q, int64_t q_stride_t, int
   if (T < 0 || W < 1) return fail(QSA_ERR_INVALID_ARG, "T must be non-negative and W positive");
   // one chunk of min(T, 64) rows of scores plus the selection state must fit
   const int64_t rows = std::min<int64_t>(T, 64);
-  if ((size_t)rows * (size_t)W * sizeof(float) + 4096 > kNoAllocScratchBytes)
+  if ((size_t)rows * (size_t)W * sizeof(float) + kPredBytes > kNoAllocScratchBytes)
     return fail(QSA_ERR_WORKSPACE,
                 "W = %d needs %lld bytes of scratch for one chunk of %lld rows; the static scratch holds %zu", W,
-                (long long)((size_t)rows * (size_t)W * sizeof(float) + 4096), (long long)rows,
+                (long long)((size_t)rows * (size_t)W * sizeof(float) + kPredBytes), (long long)rows,
                 kNoAllocScratchBytes);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -556,7 +619,7 @@ qsa_status_t qsa_mqa_prefill_topk_noalloc(const void* q, int64_t q_stride_t, int
 
 size_t qsa_prefill_topk_workspace_size(int64_t T, int32_t W) {
   if (T <= 0 || W <= 0) return 0;
-  return (size_t)T * (size_t)W * sizeof(float) + 4096;
+  return (size_t)T * (size_t)W * sizeof(float) + kPredBytes;
 }
 
 qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
@@ -575,7 +638,6 @@ qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_s
   if (!aligned(workspace, 16)) return fail(QSA_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
   // the workspace ends with the top-k kernel's per-CTA predictions, carried
   // from one chunk to the next
-  constexpr size_t kPredBytes = 4096;
   if (workspace_bytes < kPredBytes)
     return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes is too small", workspace_bytes);
   const size_t score_bytes = (workspace_bytes - kPredBytes) & ~size_t(15);

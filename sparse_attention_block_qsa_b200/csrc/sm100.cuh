@@ -183,6 +183,15 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(uint32_t M, uint32_t 
          | ((M >> 4) << 24);  // M / 16
 }
 
+// The same for fp16 A and B.
+__host__ __device__ constexpr uint32_t umma_idesc_f16_f32(uint32_t M, uint32_t N) {
+  return (1u << 4)            // D format: f32
+         | (0u << 7)          // A format: f16
+         | (0u << 10)         // B format: f16
+         | ((N >> 3) << 17)   // N / 8
+         | ((M >> 4) << 24);  // M / 16
+}
+
 // One K = 128 step of a bf16 product as eight K = 16 MMAs into d, the first
 // overwriting d.  a and b are the descriptors of the first 16-column slice of
 // the two K-major, 128-byte-swizzled operands; each holds its K columns in two

@@ -52,6 +52,19 @@ def prefill_bounds(q: torch.Tensor, k: torch.Tensor, ks: np.ndarray, W: int, sca
     """(loose, tight) tolerance arrays [rows, W] for prefill scores (column j is key ks + j)."""
     rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
     qd = _f64(q[torch.as_tensor(rows)])            # [R, 4, 128]
+    ks_r = np.asarray(ks)[rows].astype(np.int64)
+    if len(rows) and np.all(ks_r == ks_r[0]):
+        # rows that share ks see the same key window: only its W keys matter
+        k0, Nk = int(ks_r[0]), k.shape[0]
+        lo, hi = max(k0, 0), min(k0 + W, Nk)
+        loose = np.full((len(rows), W), 1e-6)
+        tight = np.full((len(rows), W), 1e-6)
+        if hi > lo:
+            kd = _f64(k[lo:hi])
+            qn = np.linalg.norm(qd, axis=-1).sum(-1)
+            loose[:, lo - k0:hi - k0] += 4e-3 * scale * qn[:, None] * np.linalg.norm(kd, axis=-1)[None, :]
+            tight[:, lo - k0:hi - k0] += TIGHT * scale * (np.abs(qd).sum(1) @ np.abs(kd).T)
+        return loose, tight
     kd = _f64(k)
     Nk = kd.shape[0]
     cols = ks[rows][:, None].astype(np.int64) + np.arange(W)[None, :]

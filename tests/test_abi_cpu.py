@@ -57,7 +57,7 @@ def decode(**kw):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(Q=5), UNSUP), (dict(Q=0), UNSUP), (dict(ps=12), UNSUP), (dict(ps=128), UNSUP),
+    (dict(Q=5), UNSUP), (dict(Q=0), UNSUP), (dict(ps=7), UNSUP), (dict(ps=1025), UNSUP),
     (dict(B=-1), INVALID), (dict(W=-1), INVALID), (dict(pages=0), INVALID), (dict(maxp=-1), INVALID),
     (dict(scale=float("nan")), INVALID), (dict(q=0), INVALID), (dict(out=0), INVALID),
     (dict(q=A + 2), ALIGN), (dict(k=A + S + 8), ALIGN), (dict(out=A + 4 * S + 2), ALIGN),
@@ -93,7 +93,7 @@ def decode_fp8(**kw):
     (dict(kscale=float("inf")), INVALID), (dict(kscale=1e30, scale=1e30), INVALID),
     (dict(krs=136), ALIGN),            # 8-byte multiple: fine for bf16 elements, not for 1-byte codes
     (dict(kps=64 * 128 + 8), ALIGN), (dict(krs=112), ALIGN), (dict(k=A + S + 8), ALIGN),
-    (dict(Q=5), UNSUP), (dict(ps=12), UNSUP), (dict(sh=100), ALIGN),
+    (dict(Q=5), UNSUP), (dict(ps=4), UNSUP), (dict(sh=100), ALIGN),
     (dict(out=A + S + 64), INVALID),   # out overlaps the 1-byte cache
 ])
 def test_decode_fp8_rejects(kw, code):

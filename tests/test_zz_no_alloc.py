@@ -65,3 +65,26 @@ def test_noalloc_rejects_rows_beyond_the_scratch():
     with pytest.raises(qsa.QSAError) as e:
         qsa.mqa_prefill_topk_noalloc(q, k, ks, ks, 65536, 16, idx=idx)
     assert e.value.status == 4
+
+
+def test_noalloc_widest_rows_fill_the_scratch_exactly():
+    # W = 65520: one chunk of 64 rows of scores plus the 4 KB of selection
+    # state fills the 16 MiB scratch exactly; the result must equal the
+    # workspace entry point's.  W = 65521 no longer fits and is refused.
+    T, W, kk = 64, 65520, 16
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(T, 4, 128, generator=g).to(torch.bfloat16).to(DEV)
+    k = torch.randn(W, 128, generator=g).to(torch.bfloat16).to(DEV)
+    ks = torch.zeros(T, dtype=torch.int32, device=DEV)
+    ke = torch.arange(T, dtype=torch.int32, device=DEV) * 3 + 40     # 40 .. 229 visible keys per row
+    ke[-1] = W                                                       # one row sees every key
+    ws = torch.empty(_abi.prefill_topk_workspace_size(T, W) // 4, dtype=torch.float32, device=DEV)
+    want = qsa.mqa_prefill_topk(q, k, ks, ke, W, kk, ws)
+    for _ in range(2):
+        got = qsa.mqa_prefill_topk_noalloc(q, k, ks, ke, W, kk)
+        torch.cuda.synchronize()
+        assert torch.equal(got, want)
+    assert qsa.device_error() == 0
+    with pytest.raises(qsa.QSAError) as e:
+        qsa.mqa_prefill_topk_noalloc(q, k, ks, ke, W + 1, kk)
+    assert e.value.status == 4

@@ -39,6 +39,10 @@ def _bind(L: C.CDLL) -> C.CDLL:
     L.qsa_oracle_topk.argtypes = [_vp, _i64, _vp, _i64, _i64, _vp, _i64, _int]
     L.qsa_oracle_e4m3_to_double.argtypes = [C.c_uint8]
     L.qsa_oracle_e4m3_to_double.restype = C.c_double
+    L.qsa_oracle_expand_indices.argtypes = [_vp, _i64, _vp, _vp, _i64, _i64, _vp, _i64]
+    L.qsa_oracle_sparse_attention.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _i64,
+                                              _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                              _vp, _f64, _vp, _vp, _int]
     L.qsa_oracle_decode_fp8.argtypes = [_vp, _i64, _i64, _i64, _vp, _f64, _i64, _i64, _i64, _i64,
                                         _vp, _i64, _i64, _vp, _i64, _i64, _f64, _vp, _i64, _int]
     return L
@@ -201,6 +205,43 @@ class Oracle:
                                           kb.shape[0], _ptr(a), _ptr(b), float(scale),
                                           _ptr(tt), _ptr(jj), tt.shape[0], _ptr(out), threads, f16)
         return out
+
+    def expand_indices(self, blocks, pos, seq_len_of_row) -> np.ndarray:
+        """Token indices [rows, 4k + 3] of selected blocks [rows, k]: four
+        tokens per block, then the row's open-group tokens, then -1."""
+        blk = _i32(blocks)
+        ps, sl = _i32(pos), _i32(seq_len_of_row)
+        rows, k = blk.shape
+        tok = np.empty((rows, 4 * k + 3), dtype=np.int32)
+        self.L.qsa_oracle_expand_indices(_ptr(blk), k, _ptr(ps), _ptr(sl), rows, k, _ptr(tok), 4 * k + 3)
+        return tok
+
+    def sparse_attention(self, q, k_cache, v_cache, page_table, row_req, row_pos, seq_lens, tok,
+                         scale: float, gate=None, threads: int = 0):
+        """Sparse core attention in fp64: q bf16 [T, Hq, 256], paged K/V bf16
+        [pages, page_size, Hkv, 256], token lists tok int32 [T, width]
+        (request-local, -1 pads) -> (out [T, Hq, 256], lse [T, Hq])."""
+        qb, qs = _bf16_bits(q)
+        kb, kst = _bf16_bits(k_cache)
+        vb, vst = _bf16_bits(v_cache)
+        if len(qs) != 3 or qs[2] != 1 or qb.shape[2] != 256:
+            raise ValueError("q must be [T, Hq, 256] with unit feature stride")
+        if kst != vst or len(kst) != 4 or kst[3] != 1 or kb.shape != vb.shape or kb.shape[3] != 256:
+            raise ValueError("K and V must be [pages, page_size, Hkv, 256] with the same strides")
+        T, Hq = qb.shape[0], qb.shape[1]
+        Hkv = kb.shape[2]
+        if Hq % Hkv:
+            raise ValueError("Hq must be a multiple of Hkv")
+        pt, rq, rp, sl, tk = _i32(page_table), _i32(row_req), _i32(row_pos), _i32(seq_lens), _i32(tok)
+        g = None if gate is None else np.ascontiguousarray(np.asarray(gate, dtype=np.float64).reshape(T, Hq))
+        out = np.empty((T, Hq, 256), dtype=np.float64)
+        lse = np.empty((T, Hq), dtype=np.float64)
+        self.L.qsa_oracle_sparse_attention(_ptr(qb), qs[0], qs[1], Hq, _ptr(kb), _ptr(vb), kb.shape[0], kb.shape[1],
+                                           kst[0], kst[1], kst[2], Hkv, _ptr(pt), pt.shape[1], pt.shape[1],
+                                           _ptr(rq), _ptr(rp), _ptr(sl), _ptr(tk), tk.shape[1], tk.shape[1], T,
+                                           None if g is None else _ptr(g), float(scale), _ptr(out), _ptr(lse),
+                                           threads)
+        return out, lse
 
     def topk(self, scores, lengths, k: int, threads: int = 0) -> np.ndarray:
         """Column indices [rows, k] of the k largest scores among each row's first

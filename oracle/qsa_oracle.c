@@ -369,3 +369,140 @@ void qsa_oracle_topk(const double *scores, int64_t stride, const int32_t *length
     topk_ctx c = {scores, stride, lengths, k, idx, idx_stride};
     parallel_for(rows, nthreads, topk_rows, &c);
 }
+
+/* ====================================================== core attention
+ *
+ * The stage after the indexer (QSA docs, MATE, section "Core Attention"):
+ * the caller keeps the top-scoring compressed blocks, expands them to token
+ * indices, and sparse attention runs over those tokens.
+ */
+
+/* Block -> token index expansion.  Row t (logical position pos[t]) keeps the
+ * blocks blk[t, 0..k); block b stands for tokens 4b .. 4b + 3.  The docs tie
+ * the widths as tokens = 4 * blocks + 3: the 3 extra slots hold the tokens of
+ * the row's open group, the tokens after its last complete group, which no
+ * compressed key covers yet: positions 4 * visible .. pos with visible =
+ * visible_blocks(pos, seq_len) (at most 3 of them).  Output row t lists, in
+ * order, the four tokens of each non-negative block index (in the order the
+ * blocks are given), then the open-group tokens ascending, then -1 up to the
+ * width 4k + 3.  A row whose position is negative keeps no open group. */
+void qsa_oracle_expand_indices(const int32_t *blk, int64_t blk_stride, const int32_t *pos,
+                               const int32_t *seq_len_of_row, int64_t rows, int64_t k,
+                               int32_t *tok, int64_t tok_stride) {
+    int64_t width = 4 * k + 3;
+    for (int64_t t = 0; t < rows; ++t) {
+        int32_t *dst = tok + t * tok_stride;
+        int64_t n = 0;
+        for (int64_t i = 0; i < k; ++i) {
+            int64_t b = blk[t * blk_stride + i];
+            if (b < 0) continue;
+            for (int64_t r = 0; r < 4; ++r) dst[n++] = (int32_t)(4 * b + r);
+        }
+        int64_t p = pos[t];
+        if (p >= 0) {
+            int64_t vis = qsa_oracle_visible_blocks(p, seq_len_of_row[t]);
+            for (int64_t j = 4 * vis; j <= p && n < width; ++j) dst[n++] = (int32_t)j;
+        }
+        while (n < width) dst[n++] = -1;
+    }
+}
+
+typedef struct {
+    const uint16_t *q; int64_t q_st, q_sh, Hq;
+    const uint16_t *k_cache, *v_cache;
+    int64_t num_pages, page_size, kv_page_stride, kv_row_stride, kv_head_stride, Hkv;
+    const int32_t *page_table; int64_t pt_stride, max_pages;
+    const int32_t *row_req, *row_pos, *seq_lens;
+    const int32_t *tok; int64_t tok_stride, width;
+    const double *gate;   /* [T, Hq] or NULL */
+    double scale;
+    double *out;          /* [T, Hq, 256] */
+    double *lse;          /* [T, Hq] */
+} sparse_attn_ctx;
+
+#define QSA_ATTN_DIM 256
+
+/* Row of token j of request r in the paged K/V pool for KV head g, or NULL
+ * when the token is outside the request or its page is missing. */
+static const uint16_t *kv_row(const sparse_attn_ctx *c, const uint16_t *cache, int64_t r, int64_t j, int64_t g) {
+    int64_t logical = j / c->page_size;
+    if (logical >= c->max_pages) return NULL;
+    int64_t page = c->page_table[r * c->pt_stride + logical];
+    if (page < 0 || page >= c->num_pages) return NULL;
+    return cache + page * c->kv_page_stride + (j % c->page_size) * c->kv_row_stride + g * c->kv_head_stride;
+}
+
+/* Softmax attention of query row t, head h, over the listed tokens that the
+ * row may see: index j >= 0, j <= pos (no future token), j < seq_len of the
+ * row's request, page present.  Each listed token counts once per listing.
+ * Scores s_i = scale * q . k_i; out = sum_i softmax(s)_i * v_i, times
+ * sigmoid(gate) when a gate is given; lse = log(sum_i exp(s_i)) (natural
+ * log).  A row with no such token gives zero output and lse = -inf.  Query
+ * heads share KV head h / (Hq / Hkv). */
+static void sparse_attn_rows(void *vctx, int64_t begin, int64_t end) {
+    sparse_attn_ctx *c = (sparse_attn_ctx *)vctx;
+    int64_t group = c->Hq / c->Hkv;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(c->width > 0 ? c->width : 1));
+    const uint16_t **vrow = (const uint16_t **)malloc(sizeof(uint16_t *) * (size_t)(c->width > 0 ? c->width : 1));
+    for (int64_t th = begin; th < end; ++th) {
+        int64_t t = th / c->Hq, h = th % c->Hq, g = h / group;
+        int64_t r = c->row_req[t], pos = c->row_pos[t];
+        double *o = c->out + th * QSA_ATTN_DIM;
+        for (int d = 0; d < QSA_ATTN_DIM; ++d) o[d] = 0.0;
+        int64_t n = 0;
+        if (r >= 0) {
+            const uint16_t *qh = c->q + t * c->q_st + h * c->q_sh;
+            for (int64_t i = 0; i < c->width; ++i) {
+                int64_t j = c->tok[t * c->tok_stride + i];
+                if (j < 0 || j > pos || j >= c->seq_lens[r]) continue;
+                const uint16_t *kr = kv_row(c, c->k_cache, r, j, g);
+                const uint16_t *vr = kv_row(c, c->v_cache, r, j, g);
+                if (!kr || !vr) continue;
+                double dot = 0.0;
+                for (int d = 0; d < QSA_ATTN_DIM; ++d) dot += bf16_to_double(qh[d]) * bf16_to_double(kr[d]);
+                s[n] = c->scale * dot;
+                vrow[n] = vr;
+                ++n;
+            }
+        }
+        if (n == 0) {
+            c->lse[th] = -INFINITY;
+            continue;
+        }
+        double m = s[0];
+        for (int64_t i = 1; i < n; ++i) m = s[i] > m ? s[i] : m;
+        double denom = 0.0;
+        for (int64_t i = 0; i < n; ++i) denom += exp(s[i] - m);
+        double lse = m + log(denom);
+        for (int64_t i = 0; i < n; ++i) {
+            double p = exp(s[i] - lse);
+            for (int d = 0; d < QSA_ATTN_DIM; ++d) o[d] += p * bf16_to_double(vrow[i][d]);
+        }
+        if (c->gate) {
+            double gt = 1.0 / (1.0 + exp(-c->gate[th]));
+            for (int d = 0; d < QSA_ATTN_DIM; ++d) o[d] *= gt;
+        }
+        c->lse[th] = lse;
+    }
+    free(s);
+    free(vrow);
+}
+
+/* Sparse core attention over paged K/V: q bf16 [T, Hq, 256] (row stride
+ * q_st, head stride q_sh), K and V bf16 [pages, page_size, Hkv, 256] with the
+ * given page, row and head strides, row t belonging to request row_req[t]
+ * (negative: a padding row) at logical position row_pos[t], token list
+ * tok[t, 0..width).  out [T, Hq, 256] and lse [T, Hq] in fp64. */
+void qsa_oracle_sparse_attention(const uint16_t *q, int64_t q_st, int64_t q_sh, int64_t Hq,
+                                 const uint16_t *k_cache, const uint16_t *v_cache, int64_t num_pages,
+                                 int64_t page_size, int64_t kv_page_stride, int64_t kv_row_stride,
+                                 int64_t kv_head_stride, int64_t Hkv,
+                                 const int32_t *page_table, int64_t pt_stride, int64_t max_pages,
+                                 const int32_t *row_req, const int32_t *row_pos, const int32_t *seq_lens,
+                                 const int32_t *tok, int64_t tok_stride, int64_t width, int64_t T,
+                                 const double *gate, double scale, double *out, double *lse, int nthreads) {
+    sparse_attn_ctx c = {q, q_st, q_sh, Hq, k_cache, v_cache, num_pages, page_size, kv_page_stride,
+                         kv_row_stride, kv_head_stride, Hkv, page_table, pt_stride, max_pages,
+                         row_req, row_pos, seq_lens, tok, tok_stride, width, gate, scale, out, lse};
+    parallel_for(T * Hq, nthreads, sparse_attn_rows, &c);
+}

@@ -538,6 +538,127 @@ def pin_f16_closed_form(orc):
     assert d[0, 0, 0] == 0.5 * (1.0 + 2.0 ** -10)
 
 
+# ---------------------------------------------------------------- core attention
+
+def pin_expand_indices_follow_cache_writer(orc):
+    """Block -> token expansion (QSA docs, "Core Attention": token width =
+    4 * blocks + 3) against the cache writer's rule: a row keeps the four
+    tokens of each selected block, then the tokens written since its last
+    complete group."""
+    rng = np.random.default_rng(31)
+    k = 4
+    rows, pos, sl, want = [], [], [], []
+    for L in range(1, 34):
+        for p in range(0, L):
+            written = keys_written_through(p)            # complete blocks at position p
+            take = sorted(rng.choice(len(written), size=min(k, len(written)), replace=False).tolist()) \
+                if written else []
+            if len(take) > 1 and rng.random() < 0.3:
+                take = take[:-1]
+            blk = take + [-1] * (k - len(take))
+            toks = [4 * b + r for b in take for r in range(4)]
+            toks += list(range(4 * len(written), p + 1))  # the open group, at most 3 tokens
+            assert len(toks) <= 4 * k + 3
+            rows.append(blk)
+            pos.append(p)
+            sl.append(L)
+            want.append(toks + [-1] * (4 * k + 3 - len(toks)))
+    rows.append([3, -1, 0, -1])                          # a padding row: blocks only
+    pos.append(-1)
+    sl.append(20)
+    want.append([12, 13, 14, 15, 0, 1, 2, 3] + [-1] * 11)
+    got = orc.expand_indices(np.array(rows), np.array(pos), np.array(sl))
+    assert np.array_equal(got, np.array(want, dtype=np.int32))
+
+
+def _attn_case(rng, lens, Hq, Hkv, ps, lo=-2, hi=2):
+    """Paged K/V pools with small-integer bf16 data, pages permuted."""
+    pages_per_req = [max(1, -(-L // ps)) for L in lens]
+    num_pages = sum(pages_per_req) + 1
+    perm = rng.permutation(num_pages)
+    table = np.full((len(lens), max(pages_per_req)), -1, dtype=np.int32)
+    at = 0
+    for r, n in enumerate(pages_per_req):
+        table[r, :n] = perm[at:at + n]
+        at += n
+    kc = int_bf16((num_pages, ps, Hkv, 256), lo, hi, rng)
+    vc = int_bf16((num_pages, ps, Hkv, 256), lo, hi, rng)
+    return kc, vc, table
+
+
+def _dense_kv(cache, table_row, ps, L):
+    """K or V of one request in token order [L, Hkv, 256] (a walk of its pages)."""
+    return torch.stack([cache[int(table_row[j // ps]), j % ps] for j in range(L)])
+
+
+def pin_sparse_attention_matches_library_sdpa(orc):
+    """When a row's list holds every token it may see (in any order, with -1
+    pads, duplicates of nothing, and future tokens that must be masked),
+    sparse attention is dense causal attention: torch's
+    scaled_dot_product_attention in fp64 on the densely gathered K/V, with the
+    grouped heads expanded, and torch.logsumexp for the LSE."""
+    rng = np.random.default_rng(32)
+    lens, Hq, Hkv, ps = [37, 70], 6, 2, 16
+    kc, vc, table = _attn_case(rng, lens, Hq, Hkv, ps)
+    rows = [(0, 36), (0, 20), (1, 69), (1, 3), (1, 0)]
+    width = 80
+    tok = np.full((len(rows), width), -1, dtype=np.int32)
+    for t, (r, p) in enumerate(rows):
+        toks = list(range(p + 1)) + list(range(p + 1, min(p + 6, lens[r])))   # some future tokens
+        toks = rng.permutation(toks).tolist()
+        slots = np.sort(rng.choice(width, size=len(toks), replace=False))
+        tok[t, slots] = toks
+    q = int_bf16((len(rows), Hq, 256), -2, 2, rng)
+    scale = 1.0 / 16.0
+    out, lse = orc.sparse_attention(q, kc, vc, table, [r for r, _ in rows], [p for _, p in rows], lens, tok,
+                                    scale=scale, threads=2)
+    group = Hq // Hkv
+    for t, (r, p) in enumerate(rows):
+        K = _dense_kv(kc, table[r], ps, p + 1).double()          # [n, Hkv, 256]
+        V = _dense_kv(vc, table[r], ps, p + 1).double()
+        Kh = K.repeat_interleave(group, dim=1).transpose(0, 1)   # [Hq, n, 256]
+        Vh = V.repeat_interleave(group, dim=1).transpose(0, 1)
+        qq = q[t].double()[:, None, :]                           # [Hq, 1, 256]
+        want = torch.nn.functional.scaled_dot_product_attention(qq, Kh, Vh, scale=scale)[:, 0]
+        want_lse = torch.logsumexp(scale * (qq @ Kh.transpose(1, 2))[:, 0], dim=-1)
+        assert np.allclose(out[t], want.numpy(), rtol=1e-12, atol=1e-12), t
+        assert np.allclose(lse[t], want_lse.numpy(), rtol=1e-12, atol=1e-12), t
+
+
+def pin_sparse_attention_closed_forms(orc):
+    rng = np.random.default_rng(33)
+    lens, Hq, Hkv, ps = [40], 4, 2, 8
+    kc, vc, table = _attn_case(rng, lens, Hq, Hkv, ps)
+    kc = torch.zeros_like(kc)                                    # every score 0: uniform weights
+    vc[..., 1, :] = vc[..., 0, :] + 100                          # KV head 1 = head 0 + 100
+    q = int_bf16((4, Hq, 256), -2, 2, rng)
+    width = 6
+    tok = np.array([[5, -1, -1, -1, -1, -1],                     # one token: out = v, lse = 0
+                    [5, 9, -1, -1, -1, -1],                      # two: the mean, lse = log 2
+                    [39, 38, -1, -1, -1, -1],                    # both after the row's position: empty
+                    [2, 3, -1, -1, -1, -1]], dtype=np.int32)     # padding row (no request)
+    req, pos = [0, 0, 0, -1], [30, 30, 30, 30]
+    gate = np.zeros((4, Hq))
+    gate[1] = 0.0
+    out, lse = orc.sparse_attention(q, kc, vc, table, req, pos, lens, tok, scale=0.5)
+    V = _dense_kv(vc, table[0], ps, 40).double().numpy()         # [40, Hkv, 256]
+    group = Hq // Hkv
+    for h in range(Hq):
+        g = h // group
+        assert np.array_equal(out[0, h], V[5, g]) and lse[0, h] == 0.0
+        assert np.array_equal(out[1, h], (V[5, g] + V[9, g]) / 2) and lse[1, h] == np.log(2.0)
+    assert np.all(out[2] == 0) and np.all(np.isneginf(lse[2]))
+    assert np.all(out[3] == 0) and np.all(np.isneginf(lse[3]))
+    # a gate of 0 halves the output exactly (sigmoid(0) = 1/2)
+    g_out, g_lse = orc.sparse_attention(q, kc, vc, table, req, pos, lens, tok, scale=0.5, gate=gate)
+    assert np.array_equal(g_out[:2], out[:2] / 2) and np.array_equal(g_lse, lse)
+    # a missing page drops its tokens: the same as leaving them out of the list
+    t2 = table.copy()
+    t2[0, 1] = -1                                                # tokens 8..15
+    m_out, _ = orc.sparse_attention(q, kc, vc, t2, req, pos, lens, tok, scale=0.5)
+    assert np.array_equal(m_out[1], out[0])                      # token 9 gone, token 5 left
+
+
 ALL_PINS = [
     pin_visible_blocks_follow_cache_writer,
     pin_decode_positions_are_last_tokens,
@@ -558,4 +679,7 @@ ALL_PINS = [
     pin_f16_decoder,
     pin_f16_matches_bf16_on_shared_values,
     pin_f16_closed_form,
+    pin_expand_indices_follow_cache_writer,
+    pin_sparse_attention_matches_library_sdpa,
+    pin_sparse_attention_closed_forms,
 ]

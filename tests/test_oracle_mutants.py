@@ -47,6 +47,19 @@ MUTANTS = {
                                       "else mag = ldexp(1.0 + man / 1024.0, ex - 14);"),
     "fp16 subnormals flushed": ("else if (ex == 0) mag = ldexp((double)man, -24);",
                                 "else if (ex == 0) mag = 0.0;"),
+    "expansion open group starts one group late": (
+        "for (int64_t j = 4 * vis; j <= p && n < width; ++j)",
+        "for (int64_t j = 4 * vis + 4; j <= p && n < width; ++j)"),
+    "expansion drops the last block token": ("for (int64_t r = 0; r < 4; ++r) dst[n++]",
+                                             "for (int64_t r = 0; r < 3; ++r) dst[n++]"),
+    "attention KV head by modulo": ("int64_t t = th / c->Hq, h = th % c->Hq, g = h / group;",
+                                    "int64_t t = th / c->Hq, h = th % c->Hq, g = h % c->Hkv;"),
+    "attention keeps future tokens": ("if (j < 0 || j > pos || j >= c->seq_lens[r]) continue;",
+                                      "if (j < 0 || j >= c->seq_lens[r]) continue;"),
+    "attention scale dropped": ("s[n] = c->scale * dot;", "s[n] = dot;"),
+    "attention gate ignored": ("double gt = 1.0 / (1.0 + exp(-c->gate[th]));", "double gt = 1.0;"),
+    "attention missing pages kept": ("if (page < 0 || page >= c->num_pages) return NULL;",
+                                     "if (page < 0) page = 0;"),
     "top-k keeps the smallest": ("if (a->v > b->v) return -1;\n    if (a->v < b->v) return 1;",
                                  "if (a->v < b->v) return -1;\n    if (a->v > b->v) return 1;"),
 }

@@ -8,8 +8,10 @@ the headline is the long-context speculative decode (16 requests, 4 query
 tokens each, log-normal contexts of 3,508-102,400 tokens, page size 64), the
 workload whose HBM roofline fraction is the decode target; the other four
 (single-request decode, 16-request decode, the 8,192-row prefill, the
-4 x 4,096-row prefill with top-512) are records under "configs", each with
-its own roofline, clocks, end-to-end and CPU-baseline figures.  `--config c`
+4 x 4,096-row prefill with top-512, and the core-attention step that follows
+the long-context decode: block -> token expansion and sparse attention over
+2,051 selected tokens per row) are records under "configs", each with its
+own roofline, clocks, end-to-end and CPU-baseline figures.  `--config c`
 times one workload only.
 
 For each workload the K timed steps are captured in one CUDA graph and
@@ -331,10 +333,133 @@ class PrefillBench:
             oracle.topk(s, np.full(s.shape[0], p.W, dtype=np.int32), wl.TOPK_K, threads=threads)
 
 
+class AttentionBench:
+    """Core-attention step after the indexer: block -> token expansion and
+    split-KV sparse attention (three launches) over one batch of selected
+    blocks; steps rotate over several selections so that they gather
+    different tokens from the 1.7 GB K/V pool."""
+    kernel = "attn_kernel"
+    bound = "hbm"
+    unit = "GB/s"
+
+    def __init__(self, cfg: int, dev: torch.device, seed: int):
+        import sparse_attention_block_qsa_b200 as qsa
+        self.qsa = qsa
+        self.inp = a = wl.make_config(cfg, seed=seed)
+        self.name = a.name
+        self.dev = dev
+        self.sets = [a.blocks] + wl.attention_block_sets(a, 3, seed + 1000)
+        self.copies = len(self.sets)
+        self.q = a.q.to(dev)
+        self.kc, self.vc = a.k_cache.to(dev), a.v_cache.to(dev)
+        self.pt, self.cu, self.sl = a.page_table.to(dev), a.cu_seqlens_q.to(dev), a.seq_lens.to(dev)
+        self.blocks = [b.to(dev) for b in self.sets]
+        k = a.blocks.shape[1]
+        self.tok = torch.empty((a.T, 4 * k + 3), dtype=torch.int32, device=dev)
+        Hq, Hkv = a.q.shape[1], a.k_cache.shape[2]
+        self.out = torch.empty((a.T, Hq, 256), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((a.T, Hq), dtype=torch.float32, device=dev)
+        ws = qsa.sparse_attention_workspace_size(a.T, Hq, Hkv, 4 * k + 3)
+        self.ws = torch.empty(ws // 4 + 4, dtype=torch.float32, device=dev)
+        self.units, self.flops, self.tokens = self._accounting(a, Hq, Hkv)
+        self.launches_per_step = 3
+        self.h2d = a.q.numel() * 2 + a.blocks.numel() * 4 + (a.cu_seqlens_q.numel() + a.seq_lens.numel()) * 4
+        self.d2h = self.out.numel() * 2 + self.lse.numel() * 4
+        self.dtype = "bf16"
+        self.config = {"workload": a.name, "requests": len(a.meta["context_tokens"]),
+                       "query_rows": a.meta["query_rows"], "heads_q_kv": list(a.meta["heads"]), "head_dim": 256,
+                       "page_size": a.meta["page_size"], "blocks_per_row": k, "tokens_per_row": 4 * k + 3,
+                       "context_tokens": a.meta["context_tokens"],
+                       "kv_pool_bytes": a.k_cache.numel() * 4, "bytes_per_step": self.units,
+                       "flop_per_step": self.flops,
+                       "l2": f"steps rotate over {self.copies} block selections; each gathers "
+                             f"{self.units / 2**20:.0f} MiB of K/V rows from a "
+                             f"{a.k_cache.numel() * 4 / 2**30:.1f} GiB pool",
+                       "e2e_inputs": "q, selected blocks and request metadata copied in each step; "
+                                     "the paged K/V cache is resident model state"}
+
+    @staticmethod
+    def _accounting(a, Hq, Hkv):
+        """Algorithmic bytes: the distinct K and V rows a request's rows
+        select (each read once), the queries, the bf16 outputs and the LSE.
+        FLOPs: 4 * 256 per (row, query head, visible token)."""
+        cu = a.cu_seqlens_q.tolist()
+        sl = a.seq_lens.tolist()
+        blocks = a.blocks.numpy()
+        uniq = 0
+        vis_tokens = 0
+        for r in range(len(sl)):
+            toks = set()
+            qlen = cu[r + 1] - cu[r]
+            for i in range(qlen):
+                t = cu[r] + i
+                pos = sl[r] - qlen + i
+                v = max(0, min((pos + 1) // 4, sl[r] // 4))
+                row = {4 * int(b) + j for b in blocks[t] if b >= 0 for j in range(4)}
+                row |= set(range(4 * v, pos + 1))
+                toks |= row
+                vis_tokens += len(row)
+            uniq += len(toks)
+        T = a.T
+        bytes_ = uniq * Hkv * 2 * 512 + T * Hq * 256 * 2 * 2 + T * Hq * 4
+        return bytes_, 4 * Hq * 256 * vis_tokens, vis_tokens
+
+    def _launch(self, blocks):
+        self.qsa.expand_block_indices(blocks, self.cu, self.sl, token_idx=self.tok)
+        self.qsa.sparse_attention(self.q, self.kc, self.vc, self.pt, self.cu, self.sl, self.tok, 1.0 / 16.0,
+                                  out=self.out, lse=self.lse, workspace=self.ws)
+
+    def step(self, i: int):
+        self._launch(self.blocks[i % self.copies])
+
+    def throughput(self, seconds_per_step: float) -> float:
+        return self.units / seconds_per_step / 1e9
+
+    def e2e_setup(self):
+        a = self.inp
+        self.host = [t.pin_memory() for t in (a.q, a.cu_seqlens_q, a.seq_lens)]
+        self.host_blocks = [b.pin_memory() for b in self.sets]
+        self.host_out = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
+        self.host_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step(self, i: int):
+        for dst, src in zip((self.q, self.cu, self.sl), self.host):
+            dst.copy_(src, non_blocking=True)
+        b = self.blocks[i % self.copies]
+        b.copy_(self.host_blocks[i % self.copies], non_blocking=True)
+        self._launch(b)
+        self.host_out.copy_(self.out, non_blocking=True)
+        self.host_lse.copy_(self.lse, non_blocking=True)
+
+    def oracle_sample(self):
+        return 8 / self.inp.T, "8 query rows (two requests), all 24 heads (scaled to the full batch)"
+
+    def oracle_step(self, threads: int = 0):
+        import oracle
+        a = self.inp
+        rows = slice(0, 8)
+        cu = a.cu_seqlens_q.tolist()
+        sl = a.seq_lens.tolist()
+        req, pos, ln = [], [], []
+        for r in range(2):
+            qlen = cu[r + 1] - cu[r]
+            for i in range(qlen):
+                req.append(r)
+                pos.append(oracle.logical_position(sl[r], qlen, i))
+                ln.append(sl[r])
+        tok = oracle.expand_indices(a.blocks[rows].numpy(), pos, ln)
+        oracle.sparse_attention(a.q[rows], a.k_cache, a.v_cache, a.page_table, req, pos, a.seq_lens, tok,
+                                scale=1.0 / 16.0, threads=threads)
+
+
 def make_bench(cfg: int, dev, seed: int, fp8: bool = False):
     if fp8 and cfg not in (1, 2, 3):
         raise ValueError("the fp8 key cache applies to the decode configurations 1-3")
-    return DecodeBench(cfg, dev, seed, fp8) if cfg in (1, 2, 3) else PrefillBench(cfg, dev, seed)
+    if cfg in (1, 2, 3):
+        return DecodeBench(cfg, dev, seed, fp8)
+    if cfg == 6:
+        return AttentionBench(cfg, dev, seed)
+    return PrefillBench(cfg, dev, seed)
 
 
 # ------------------------------------------------------------------ timing
@@ -445,7 +570,7 @@ def cpu_baseline(b, budget_s: float = 10.0) -> dict:
 # ------------------------------------------------------------------ main
 
 HEADLINE = 3            # the long-context spec-decode workload: the decode roofline target
-ALL_CONFIGS = [3, 1, 2, 4, 5]
+ALL_CONFIGS = [3, 1, 2, 4, 5, 6]
 
 
 def run_reference(args, rank: int, world: int):
@@ -482,7 +607,12 @@ class _HostOnly:
         self.inp = wl.make_config(cfg)
         self.fp8 = fp8 and cfg in (1, 2, 3)
         self.k_scale = 1.0
-        if cfg in (1, 2, 3):
+        if cfg == 6:
+            a = self.inp
+            self.units, _, _ = AttentionBench._accounting(a, a.q.shape[1], a.k_cache.shape[2])
+            self.unit = "GB/s"
+            self.config = {"workload": a.name, "query_rows": a.meta["query_rows"], "blocks_per_row": a.blocks.shape[1]}
+        elif cfg in (1, 2, 3):
             d = self.inp
             if self.fp8:
                 d.k_cache, self.k_scale = wl.e4m3_cache(d.k_cache)
@@ -503,12 +633,16 @@ class _HostOnly:
         return self.units / s / (1e9 if self.unit == "GB/s" else 1e12)
 
     def oracle_sample(self):
+        if self.cfg == 6:
+            return AttentionBench.oracle_sample(self)
         if self.cfg in (1, 2, 3):
             return 1.0, "one full step (every score of the batch)"
         return 64 / self.inp.T, "64 query rows of the batch, every column (scaled to the full batch)"
 
     def oracle_step(self, threads):
-        if self.cfg in (1, 2, 3):
+        if self.cfg == 6:
+            AttentionBench.oracle_step(self, threads)
+        elif self.cfg in (1, 2, 3):
             DecodeBench.oracle_step(self, threads)
         else:
             PrefillBench.oracle_step(self, threads)
@@ -614,7 +748,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=None, choices=[1, 2, 3, 4, 5],
+    ap.add_argument("--config", type=int, default=None, choices=[1, 2, 3, 4, 5, 6],
                     help="one workload only (default: all five, the long-context spec-decode one as the headline)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -286,6 +286,73 @@ qsa_status_t qsa_mqa_prefill_topk_noalloc(const void* q, int64_t q_stride_t, int
                                           int64_t T, float scale, int32_t W, int32_t topk_k, int32_t* idx,
                                           int64_t idx_stride, void* stream);
 
+/*
+ * qsa_expand_block_indices - selected compressed blocks to token indices.
+ *
+ * The step between top-k selection and core attention (QSA docs, MATE,
+ * section "Core Attention": with a block hint the token list is
+ * 4 * blocks + 3 wide, at most 4 * 512 + 3 = 2051 tokens).  Block b stands
+ * for request-local tokens 4b .. 4b + 3; the 3 extra slots hold the row's
+ * open group, the tokens after its last complete 4-token group (positions
+ * 4 * visible .. pos, at most 3), which no compressed key covers yet.
+ *
+ *   blocks       int32 [T, k], row stride blk_stride (>= k when T > 1);
+ *                negative entries are skipped (padding).  1 <= k <= 512.
+ *   cu_seqlens_q int32 [R + 1], seq_lens int32 [R]: query rows of request r
+ *                are cu_seqlens_q[r] .. cu_seqlens_q[r+1] - 1, row i of it at
+ *                logical position seq_lens[r] - qlen_r + i (vLLM qsa_cache.py,
+ *                "_logical_positions").  cu_seqlens_q[R] == T.
+ *   token_idx    int32 [T, 4k + 3] output, row stride tok_stride: the four
+ *                tokens of each non-negative block in the given order, then
+ *                the open-group tokens ascending, then -1.
+ */
+qsa_status_t qsa_expand_block_indices(const int32_t* blocks, int64_t blk_stride, int32_t k,
+                                      const int32_t* cu_seqlens_q, const int32_t* seq_lens, int32_t R, int64_t T,
+                                      int32_t* token_idx, int64_t tok_stride, void* stream);
+
+/*
+ * qsa_sparse_attention - sparse core attention over selected tokens of a
+ * paged K/V cache (QSA docs, MATE, section "Core Attention": request-local
+ * token indices shared by all query heads, -1 pads, invalid and future
+ * tokens masked, paged K/V [pages, page_size, Hkv, 256], optional sigmoid
+ * gate, natural-log LSE; empty selections give zero output and -inf LSE).
+ *
+ * For query row t of request r (at logical position pos, as in
+ * qsa_expand_block_indices) and query head h (KV head g = h / (Hq / Hkv)),
+ * over the listed tokens j with 0 <= j <= pos, j < seq_lens[r] and a valid
+ * page (page_table[r, j / page_size] in [0, num_pages)), each listed
+ * occurrence counting once:
+ *     s_j = scale * q[t, h] . K[j, g],   out[t, h] = sum_j softmax(s)_j V[j, g]
+ * times sigmoid(gate[t, h]) when gate is given; lse[t, h] = log(sum_j e^s_j).
+ *
+ *   q          bf16 [T, Hq, 256]: row stride q_stride_t, head stride
+ *              q_stride_h (>= 256), multiples of 8; 16-byte aligned.
+ *   k_cache,   bf16 [num_pages, page_size, Hkv, 256] with the given page,
+ *   v_cache    row and head strides (elements, multiples of 8); 16-byte
+ *              aligned.  Hq a multiple of Hkv, Hq / Hkv <= 16 (24 / 2 is the
+ *              QSA geometry).
+ *   page_table int32 [R, max_pages], row stride pt_stride.
+ *   token_idx  int32 [T, width], row stride tok_stride (>= width).
+ *   gate       fp32 [T, Hq] or NULL.   scale: softmax scale (finite).
+ *   out        bf16 [T, Hq, 256], row stride out_stride_t (>= Hq * 256),
+ *              heads contiguous; 16-byte aligned; must not overlap inputs.
+ *   lse        fp32 [T, Hq] or NULL.
+ *   workspace  16-byte aligned, qsa_sparse_attention_workspace_size(T, Hq,
+ *              Hkv, width) bytes (split-KV partial results); smaller returns
+ *              QSA_ERR_WORKSPACE.
+ * Two launches on `stream`: the split-KV attention and the merge of splits.
+ */
+qsa_status_t qsa_sparse_attention(const void* q, int64_t q_stride_t, int64_t q_stride_h, int32_t Hq,
+                                  const void* k_cache, const void* v_cache, int64_t num_pages, int32_t page_size,
+                                  int64_t kv_page_stride, int64_t kv_row_stride, int64_t kv_head_stride, int32_t Hkv,
+                                  const int32_t* page_table, int64_t pt_stride, int32_t max_pages,
+                                  const int32_t* cu_seqlens_q, const int32_t* seq_lens, int32_t R,
+                                  const int32_t* token_idx, int64_t tok_stride, int32_t width, int64_t T,
+                                  const float* gate, float scale, void* out, int64_t out_stride_t, float* lse,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+size_t qsa_sparse_attention_workspace_size(int64_t T, int32_t Hq, int32_t Hkv, int32_t width);
+
 #ifdef __cplusplus
 }
 #endif

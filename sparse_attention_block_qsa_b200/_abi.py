@@ -41,6 +41,11 @@ SIGNATURES = {
     "qsa_prefill_topk_workspace_size": (_sz, [_i64, _i32]),
     "qsa_mqa_prefill_topk_noalloc": (C.c_int, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f32, _i32,
                                                _i32, _vp, _i64, _vp]),
+    "qsa_expand_block_indices": (C.c_int, [_vp, _i64, _i32, _vp, _vp, _i32, _i64, _vp, _i64, _vp]),
+    "qsa_sparse_attention": (C.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _i64, _i32, _i64, _i64, _i64, _i32,
+                                       _vp, _i64, _i32, _vp, _vp, _i32, _vp, _i64, _i32, _i64, _vp, _f32,
+                                       _vp, _i64, _vp, _vp, _sz, _vp]),
+    "qsa_sparse_attention_workspace_size": (_sz, [_i64, _i32, _i32, _i32]),
 }
 
 STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_ALIGNMENT", 3: "QSA_ERR_UNSUPPORTED",
@@ -276,3 +281,88 @@ def mqa_prefill_topk_noalloc(q: torch.Tensor, k: torch.Tensor, ks: torch.Tensor,
         _ptr(q), q.stride(0), q.stride(1), _ptr(k), k.stride(0), k.shape[0], _ptr(ks), _ptr(ke), T, scale, W,
         topk_k, _ptr(idx), idx.stride(0), _stream(stream)))
     return idx
+
+
+def _index_checks(cu_seqlens_q, seq_lens):
+    for t, n in ((cu_seqlens_q, "cu_seqlens_q"), (seq_lens, "seq_lens")):
+        _need(t, n, torch.int32, 1)
+        if t.stride(0) != 1:
+            raise ValueError(f"{n} must be contiguous")
+    if cu_seqlens_q.shape[0] != seq_lens.shape[0] + 1:
+        raise ValueError("cu_seqlens_q must have one more entry than seq_lens")
+
+
+def expand_block_indices(blocks: torch.Tensor, cu_seqlens_q: torch.Tensor, seq_lens: torch.Tensor,
+                         token_idx: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Selected blocks int32 [T, k] -> token indices int32 [T, 4k + 3] (four
+    tokens per block, then the row's open group, then -1)."""
+    _need(blocks, "blocks", torch.int32, 2)
+    _index_checks(cu_seqlens_q, seq_lens)
+    if blocks.stride(1) != 1:
+        raise ValueError("blocks need a unit column stride")
+    T, k = blocks.shape
+    if token_idx is None:
+        token_idx = torch.empty((T, 4 * k + 3), dtype=torch.int32, device=blocks.device)
+    _need(token_idx, "token_idx", torch.int32, 2)
+    if token_idx.shape != (T, 4 * k + 3) or token_idx.stride(1) != 1:
+        raise ValueError("token_idx must be [T, 4k + 3] with unit column stride")
+    _check("qsa_expand_block_indices", lib().qsa_expand_block_indices(
+        _ptr(blocks), blocks.stride(0), k, _ptr(cu_seqlens_q), _ptr(seq_lens), seq_lens.shape[0], T,
+        _ptr(token_idx), token_idx.stride(0), _stream(stream)))
+    return token_idx
+
+
+def sparse_attention_workspace_size(T: int, Hq: int, Hkv: int, width: int) -> int:
+    return int(lib().qsa_sparse_attention_workspace_size(T, Hq, Hkv, width))
+
+
+def sparse_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
+                     cu_seqlens_q: torch.Tensor, seq_lens: torch.Tensor, token_idx: torch.Tensor, scale: float,
+                     gate: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                     lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """Sparse core attention: q bf16 [T, Hq, 256], K/V bf16 [pages, page_size,
+    Hkv, 256], token_idx int32 [T, width] -> (out bf16 [T, Hq, 256], lse fp32
+    [T, Hq]).  The workspace (any CUDA tensor, 16-byte aligned) is allocated
+    here by torch when not given."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(page_table, "page_table", torch.int32, 2)
+    _need(token_idx, "token_idx", torch.int32, 2)
+    _index_checks(cu_seqlens_q, seq_lens)
+    T, Hq, Dq = q.shape
+    if Dq != 256 or q.stride(2) != 1:
+        raise ValueError("q must be [T, Hq, 256] with unit feature stride")
+    if k_cache.shape != v_cache.shape or k_cache.stride() != v_cache.stride() or k_cache.shape[3] != 256 \
+            or k_cache.stride(3) != 1:
+        raise ValueError("k_cache and v_cache must be [pages, page_size, Hkv, 256] with the same strides")
+    if token_idx.shape[0] != T or token_idx.stride(1) != 1 or page_table.stride(1) != 1:
+        raise ValueError("token_idx must be [T, width] and page_table [R, max_pages], unit column strides")
+    if page_table.shape[0] != seq_lens.shape[0]:
+        raise ValueError("page_table needs one row per request")
+    Hkv = k_cache.shape[2]
+    width = token_idx.shape[1]
+    if gate is not None:
+        _need(gate, "gate", torch.float32, 2)
+        if gate.shape != (T, Hq) or not gate.is_contiguous():
+            raise ValueError("gate must be contiguous fp32 [T, Hq]")
+    if out is None:
+        out = torch.empty((T, Hq, 256), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, 3)
+    if out.shape != (T, Hq, 256) or out.stride(2) != 1 or out.stride(1) != 256:
+        raise ValueError("out must be [T, Hq, 256] with contiguous heads")
+    if lse is None:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    _need(lse, "lse", torch.float32, 2)
+    if lse.shape != (T, Hq) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [T, Hq]")
+    need = sparse_attention_workspace_size(T, Hq, Hkv, max(width, 1))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16) // 4 + 4, dtype=torch.float32, device=q.device)
+    _check("qsa_sparse_attention", lib().qsa_sparse_attention(
+        _ptr(q), q.stride(0), q.stride(1), Hq, _ptr(k_cache), _ptr(v_cache), k_cache.shape[0], k_cache.shape[1],
+        k_cache.stride(0), k_cache.stride(1), k_cache.stride(2), Hkv, _ptr(page_table), page_table.stride(0),
+        page_table.shape[1], _ptr(cu_seqlens_q), _ptr(seq_lens), seq_lens.shape[0], _ptr(token_idx),
+        token_idx.stride(0), width, T, _ptr(gate), float(scale), _ptr(out), out.stride(0), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, lse

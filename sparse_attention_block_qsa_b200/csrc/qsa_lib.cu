@@ -16,6 +16,7 @@
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "topk.cuh"
+#include "attention.cuh"
 
 namespace {
 
@@ -136,6 +137,7 @@ qsa_status_t device_info(int* sms) {
         {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::E4M3, true>), qsa::decode::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel<false>), qsa::prefill::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel<true>), qsa::prefill::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::attn::attn_kernel), qsa::attn::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_rows_kernel), qsa::topk::ROWS_SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_stream_kernel), qsa::topk::STREAM_SMEM_BYTES},
     };
@@ -354,6 +356,20 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 void* g_noalloc_ptr[kMaxDevices];
 std::mutex g_noalloc_mu;
+
+// Split-KV plan of the sparse attention: a row's token list is cut into
+// `splits` runs of `cps` 32-entry chunks, so that rows x KV heads x splits
+// gives the grid about 8 CTAs per SM of a 148-SM part (device independent,
+// so the workspace size depends on the shapes only).
+void attn_splits(int64_t T, int32_t Hkv, int32_t width, int32_t* splits, int32_t* cps) {
+  const int64_t chunks = std::max<int64_t>(1, ((int64_t)width + qsa::attn::CHUNK - 1) / qsa::attn::CHUNK);
+  const int64_t pairs = std::max<int64_t>(1, T * Hkv);
+  int64_t sp = std::min<int64_t>(chunks, std::max<int64_t>(1, (1184 + pairs - 1) / pairs));
+  const int64_t per = (chunks + sp - 1) / sp;
+  sp = (chunks + per - 1) / per;
+  *splits = (int32_t)sp;
+  *cps = (int32_t)per;
+}
 
 }  // namespace
 
@@ -682,6 +698,145 @@ qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_s
     if (st != QSA_OK) return st;
   }
   return ok();
+}
+
+qsa_status_t qsa_expand_block_indices(const int32_t* blocks, int64_t blk_stride, int32_t k, const int32_t* cu_seqlens_q,
+                                      const int32_t* seq_lens, int32_t R, int64_t T, int32_t* token_idx,
+                                      int64_t tok_stride, void* stream) {
+  if (T < 0 || R < 0) return fail(QSA_ERR_INVALID_ARG, "T and R must be non-negative");
+  if (k < 1 || k > 512) return fail(QSA_ERR_UNSUPPORTED, "k = %d blocks per row; 1..512 supported", k);
+  if (T == 0) return ok();
+  if (R == 0) return fail(QSA_ERR_INVALID_ARG, "T > 0 rows need at least one request");
+  if (T > INT32_MAX) return fail(QSA_ERR_UNSUPPORTED, "T = %lld rows exceeds 2^31 - 1", (long long)T);
+  if (!blocks || !cu_seqlens_q || !seq_lens || !token_idx) return fail(QSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(blocks, 4) || !aligned(token_idx, 4) || !aligned(cu_seqlens_q, 4) || !aligned(seq_lens, 4))
+    return fail(QSA_ERR_ALIGNMENT, "index arrays must be 4-byte aligned");
+  const int64_t width = 4 * (int64_t)k + 3;
+  if (T > 1 && (blk_stride < k || tok_stride < width))
+    return fail(QSA_ERR_INVALID_ARG, "blk_stride must be >= k and tok_stride >= 4k + 3");
+  if (overlaps(span(token_idx, 4, T, tok_stride, 1, 0, 1, 0, width), span(blocks, 4, T, blk_stride, 1, 0, 1, 0, k)))
+    return fail(QSA_ERR_INVALID_ARG, "token_idx overlaps blocks");
+  int sms = 0;
+  qsa_status_t st = device_info(&sms);
+  if (st != QSA_OK) return st;
+  qsa::attn::ExpandParams p{blocks, T > 1 ? blk_stride : k, k, cu_seqlens_q, seq_lens, R, T, token_idx,
+                            T > 1 ? tok_stride : width};
+  const int64_t blocks_n = (T * 32 + 255) / 256;
+  qsa::attn::expand_kernel<<<(unsigned)blocks_n, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status("index expansion kernel");
+}
+
+size_t qsa_sparse_attention_workspace_size(int64_t T, int32_t Hq, int32_t Hkv, int32_t width) {
+  if (T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || width <= 0) return 0;
+  int32_t splits = 0, cps = 0;
+  attn_splits(T, Hkv, width, &splits, &cps);
+  const size_t group = (size_t)(Hq / Hkv);
+  return (size_t)T * (size_t)Hkv * (size_t)splits * group * (qsa::attn::D + 2) * sizeof(float);
+}
+
+qsa_status_t qsa_sparse_attention(const void* q, int64_t q_stride_t, int64_t q_stride_h, int32_t Hq, const void* k_cache,
+                                  const void* v_cache, int64_t num_pages, int32_t page_size, int64_t kv_page_stride,
+                                  int64_t kv_row_stride, int64_t kv_head_stride, int32_t Hkv,
+                                  const int32_t* page_table, int64_t pt_stride, int32_t max_pages,
+                                  const int32_t* cu_seqlens_q, const int32_t* seq_lens, int32_t R,
+                                  const int32_t* token_idx, int64_t tok_stride, int32_t width, int64_t T,
+                                  const float* gate, float scale, void* out, int64_t out_stride_t, float* lse,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  using qsa::attn::D;
+  if (T < 0 || R < 0 || width < 0 || max_pages < 0) return fail(QSA_ERR_INVALID_ARG, "negative size argument");
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > qsa::attn::MAX_GROUP)
+    return fail(QSA_ERR_UNSUPPORTED, "Hq = %d, Hkv = %d: Hq must be a multiple of Hkv with at most %d query heads per KV head",
+                Hq, Hkv, qsa::attn::MAX_GROUP);
+  if (page_size < 1) return fail(QSA_ERR_INVALID_ARG, "page_size must be positive");
+  if (num_pages < 1 || num_pages > INT32_MAX) return fail(QSA_ERR_INVALID_ARG, "num_pages out of range");
+  if (!std::isfinite(scale)) return fail(QSA_ERR_INVALID_ARG, "scale must be finite");
+  if (T == 0) return ok();
+  if (T > INT32_MAX) return fail(QSA_ERR_UNSUPPORTED, "T = %lld rows exceeds 2^31 - 1", (long long)T);
+  if (R == 0) return fail(QSA_ERR_INVALID_ARG, "T > 0 rows need at least one request");
+  if (!q || !k_cache || !v_cache || !cu_seqlens_q || !seq_lens || !out || (width > 0 && !token_idx) ||
+      (max_pages > 0 && !page_table))
+    return fail(QSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
+    return fail(QSA_ERR_ALIGNMENT, "q, k_cache, v_cache and out must be 16-byte aligned");
+  if ((gate && !aligned(gate, 4)) || (lse && !aligned(lse, 4)) || (token_idx && !aligned(token_idx, 4)) ||
+      (page_table && !aligned(page_table, 4)))
+    return fail(QSA_ERR_ALIGNMENT, "gate, lse, token_idx and page_table must be 4-byte aligned");
+  const int64_t strides[6] = {T > 1 ? q_stride_t : 8, Hq > 1 ? q_stride_h : 8, num_pages > 1 ? kv_page_stride : 8,
+                              page_size > 1 ? kv_row_stride : 8, Hkv > 1 ? kv_head_stride : 8,
+                              T > 1 ? out_stride_t : 8};
+  for (int i = 0; i < 6; ++i)
+    if (strides[i] <= 0 || strides[i] % 8 != 0)
+      return fail(QSA_ERR_ALIGNMENT, "strides must be positive multiples of 8 elements (got %lld)", (long long)strides[i]);
+  if (Hq > 1 && q_stride_h < D) return fail(QSA_ERR_INVALID_ARG, "q_stride_h below the head dimension 256");
+  if (Hkv > 1 && kv_head_stride < D) return fail(QSA_ERR_INVALID_ARG, "kv_head_stride below 256");
+  if (page_size > 1 && kv_row_stride < (int64_t)Hkv * (Hkv > 1 ? kv_head_stride : D))
+    return fail(QSA_ERR_INVALID_ARG, "kv_row_stride too small for Hkv heads");
+  if (T > 1 && out_stride_t < (int64_t)Hq * D) return fail(QSA_ERR_INVALID_ARG, "out_stride_t below Hq * 256");
+  if (T > 1 && width > 0 && tok_stride < width) return fail(QSA_ERR_INVALID_ARG, "tok_stride below width");
+  if (max_pages > 0 && R > 1 && pt_stride < max_pages) return fail(QSA_ERR_INVALID_ARG, "pt_stride below max_pages");
+  {
+    const Range ro = span(out, 2, T, T > 1 ? out_stride_t : 0, Hq, D, 1, 0, D);
+    bool bad = overlaps(ro, span(q, 2, T, T > 1 ? q_stride_t : 0, Hq, Hq > 1 ? q_stride_h : 0, 1, 0, D));
+    const Range rk = span(k_cache, 2, num_pages, num_pages > 1 ? kv_page_stride : 0, page_size,
+                          page_size > 1 ? kv_row_stride : 0, Hkv, Hkv > 1 ? kv_head_stride : 0, D);
+    const Range rv = span(v_cache, 2, num_pages, num_pages > 1 ? kv_page_stride : 0, page_size,
+                          page_size > 1 ? kv_row_stride : 0, Hkv, Hkv > 1 ? kv_head_stride : 0, D);
+    bad = bad || overlaps(ro, rk) || overlaps(ro, rv);
+    if (lse) bad = bad || overlaps(span(lse, 4, T, Hq, 1, 0, 1, 0, Hq), ro);
+    if (bad) return fail(QSA_ERR_INVALID_ARG, "out overlaps an input (or lse)");
+  }
+  int32_t splits = 1, cps = 1;
+  attn_splits(T, Hkv, width, &splits, &cps);
+  const size_t need = qsa_sparse_attention_workspace_size(T, Hq, Hkv, width > 0 ? width : 1);
+  if (!workspace || workspace_bytes < need)
+    return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes; %zu needed", workspace_bytes, need);
+  if (!aligned(workspace, 16)) return fail(QSA_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  int sms = 0;
+  qsa_status_t st = device_info(&sms);
+  if (st != QSA_OK) return st;
+  qsa::attn::Params p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.q_st = q_stride_t;
+  p.q_sh = q_stride_h;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.k = static_cast<const uint16_t*>(k_cache);
+  p.v = static_cast<const uint16_t*>(v_cache);
+  p.num_pages = num_pages;
+  p.page_size = page_size;
+  p.kv_page_stride = kv_page_stride;
+  p.kv_row_stride = kv_row_stride;
+  p.kv_head_stride = kv_head_stride;
+  p.page_table = page_table;
+  p.pt_stride = pt_stride;
+  p.max_pages = max_pages;
+  p.cu = cu_seqlens_q;
+  p.seq_lens = seq_lens;
+  p.R = R;
+  p.tok = token_idx;
+  p.tok_stride = T > 1 ? tok_stride : width;
+  p.width = width;
+  p.T = T;
+  p.splits = splits;
+  p.chunks_per_split = cps;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  float* ws = static_cast<float*>(workspace);
+  p.part_o = ws;
+  p.part_ml = ws + (size_t)T * Hkv * splits * p.group * D;
+  p.gate = gate;
+  p.out = static_cast<uint16_t*>(out);
+  p.out_st = T > 1 ? out_stride_t : (int64_t)Hq * D;
+  p.lse = lse;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t ctas = T * Hkv * splits;
+  if (ctas > INT32_MAX) return fail(QSA_ERR_UNSUPPORTED, "too many rows for one launch");
+  qsa::attn::attn_kernel<<<(unsigned)ctas, qsa::attn::THREADS, qsa::attn::SMEM_BYTES, s>>>(p);
+  st = launch_status("sparse attention kernel");
+  if (st != QSA_OK) return st;
+  const int64_t warps = T * Hq;
+  qsa::attn::combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(p);
+  return launch_status("sparse attention combine kernel");
 }
 
 }  // extern "C"

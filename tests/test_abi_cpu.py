@@ -206,3 +206,54 @@ def test_oracle_fp8_accepts_float8_and_uint8_views():
 def test_selftest_rejects_long_limit():
     L = qsa.lib()
     assert L.qsa_selftest_bounded_wait(20_000_000_000, 0, None) == INVALID, L.qsa_last_error_detail().decode()
+
+
+def attention(**kw):
+    a = dict(q=A, qst=24 * 256, qsh=256, Hq=24, k=A + S, v=A + 2 * S, pages=100, ps=64, kps=64 * 512, krs=512,
+             khs=256, Hkv=2, pt=A + 3 * S, pts=10, maxp=10, cu=A + 4 * S, sl=A + 4 * S + 4096, R=4, tok=A + 5 * S,
+             toks=2051, width=2051, T=16, gate=None, scale=0.0625, out=A + 6 * S, ost=24 * 256, lse=None,
+             ws=A + 7 * S, wsb=1 << 30)
+    a.update(kw)
+    L = qsa.lib()
+    st = L.qsa_sparse_attention(a["q"], a["qst"], a["qsh"], a["Hq"], a["k"], a["v"], a["pages"], a["ps"], a["kps"],
+                                a["krs"], a["khs"], a["Hkv"], a["pt"], a["pts"], a["maxp"], a["cu"], a["sl"], a["R"],
+                                a["tok"], a["toks"], a["width"], a["T"], a["gate"], a["scale"], a["out"], a["ost"],
+                                a["lse"], a["ws"], a["wsb"], None)
+    return st, L.qsa_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=25), UNSUP), (dict(Hq=34, Hkv=2), UNSUP), (dict(Hkv=0), UNSUP), (dict(T=-1), INVALID),
+    (dict(ps=0), INVALID), (dict(pages=0), INVALID), (dict(scale=float("inf")), INVALID), (dict(R=0), INVALID),
+    (dict(q=0), INVALID), (dict(out=0), INVALID), (dict(tok=0), INVALID),
+    (dict(q=A + 8), ALIGN), (dict(k=A + S + 2), ALIGN), (dict(out=A + 6 * S + 4), ALIGN),
+    (dict(qsh=100), ALIGN), (dict(krs=500), ALIGN), (dict(qsh=128), INVALID), (dict(khs=128), INVALID),
+    (dict(krs=256), INVALID), (dict(ost=256), INVALID), (dict(toks=100), INVALID), (dict(pts=5), INVALID),
+    (dict(out=A + 112), INVALID),                      # out overlaps q
+    (dict(wsb=1024), WS), (dict(ws=0), WS),
+])
+def test_attention_rejects(kw, code):
+    st, detail = attention(**kw)
+    assert st == code, detail
+    assert detail
+
+
+def test_attention_workspace_size():
+    n = qsa.sparse_attention_workspace_size(64, 24, 2, 2051)
+    # 64 rows x 2 KV heads = 128 pairs -> ceil(1184 / 128) = 10 splits of ceil(65 / 10) = 7
+    # of the 65 chunks of 32 entries; 12 heads x (256 + 2) floats per split
+    assert n == 64 * 2 * 10 * 12 * 258 * 4
+    assert qsa.sparse_attention_workspace_size(0, 24, 2, 2051) == 0
+    assert qsa.sparse_attention_workspace_size(4, 24, 5, 2051) == 0
+
+
+@pytest.mark.parametrize("kw,code", [(dict(k=0), UNSUP), (dict(k=513), UNSUP), (dict(T=-1), INVALID),
+                                     (dict(R=0), INVALID), (dict(blk=0), INVALID), (dict(tok=A + 2), ALIGN),
+                                     (dict(tks=10), INVALID), (dict(tok=A + 4), INVALID)])
+def test_expand_rejects(kw, code):
+    a = dict(blk=A, bs=512, k=512, cu=A + S, sl=A + S + 4096, R=4, T=16, tok=A + 2 * S, tks=2051)
+    a.update(kw)
+    L = qsa.lib()
+    st = L.qsa_expand_block_indices(a["blk"], a["bs"], a["k"], a["cu"], a["sl"], a["R"], a["T"], a["tok"], a["tks"],
+                                    None)
+    assert st == code, L.qsa_last_error_detail().decode()

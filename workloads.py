@@ -206,8 +206,32 @@ CONFIG_NAMES = {
     3: "specdecode_b16_q4_ctx3508-102400_ps64",
     4: "prefill_t8192_prefix50144",
     5: "prefill_4x4096_prefix102400_top512",
+    6: "core_attention_b16_q4_top512_h24x2_d256_ps64",
 }
 TOPK_K = 512
+
+
+def attention_block_sets(a: "AttentionInputs", n: int, seed: int) -> list:
+    """n more block selections for the rows of ``a`` (the same rule as
+    make_attention: k visible blocks per row uniformly without replacement,
+    ascending, -1 padded), so that repeated steps gather different tokens."""
+    g = _gen(seed)
+    cu = a.cu_seqlens_q.tolist()
+    sl = a.seq_lens.tolist()
+    k = a.blocks.shape[1]
+    out = []
+    for _ in range(n):
+        blocks = torch.full_like(a.blocks, -1)
+        for r in range(len(sl)):
+            qlen = cu[r + 1] - cu[r]
+            for i in range(qlen):
+                pos = sl[r] - qlen + i
+                vis = max(0, min((pos + 1) // TOKENS_PER_KEY, sl[r] // TOKENS_PER_KEY))
+                m = min(k, vis)
+                if m:
+                    blocks[cu[r] + i, :m] = torch.randperm(vis, generator=g)[:m].sort().values.to(torch.int32)
+        out.append(blocks)
+    return out
 
 
 def make_config(idx: int, seed: int = 0):
@@ -224,4 +248,75 @@ def make_config(idx: int, seed: int = 0):
         return make_prefill(name, [8192], [50144], seed=seed)
     if idx == 5:
         return make_prefill(name, [4096] * 4, [102400] * 4, seed=seed)
+    if idx == 6:
+        # the core-attention step after workload 3's indexer: the same 16
+        # requests and 4 query rows each, top-512 blocks (2,051 tokens per row),
+        # 24 query heads over 2 KV heads of dimension 256, 64-token pages
+        ctx = lognormal_contexts(16, 3508, 102400, 16 * 51200, seed)
+        return make_attention(name, ctx, [4] * 16, 24, 2, 64, TOPK_K, seed=seed)
     raise KeyError(idx)
+
+
+@dataclass
+class AttentionInputs:
+    """Sparse core-attention inputs (all tensors on the CPU): query rows of R
+    requests packed by ``cu_seqlens_q``, paged K and V pools, and the selected
+    compressed blocks of every row (ascending, -1 padded)."""
+    name: str
+    q: torch.Tensor            # bf16 [T, Hq, 256]
+    k_cache: torch.Tensor      # bf16 [pages, page_size, Hkv, 256]
+    v_cache: torch.Tensor      # bf16 [pages, page_size, Hkv, 256]
+    page_table: torch.Tensor   # int32 [R, max_pages]
+    cu_seqlens_q: torch.Tensor # int32 [R + 1]
+    seq_lens: torch.Tensor     # int32 [R]
+    blocks: torch.Tensor       # int32 [T, k]
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def T(self) -> int:
+        return self.q.shape[0]
+
+
+ATTN_DIM = 256     # core attention head dimension (QSA docs, "Core Attention": D256)
+
+
+def make_attention(name: str, seq_lens: list[int], qlens: list[int], Hq: int, Hkv: int, page_size: int,
+                   k: int, seed: int, spare_pages: int = 1) -> AttentionInputs:
+    """Paged K/V pools with N(0, 1) bf16 rows (pages handed out by a random
+    permutation, -1 past a request's pages), N(0, 1) queries, and for every
+    query row k block indices drawn uniformly without replacement from the
+    blocks the row can see (fewer when it sees fewer), ascending, -1 padded.
+    Row i of request r sits at position seq_lens[r] - qlens[r] + i."""
+    g = _gen(seed)
+    R = len(seq_lens)
+    pages_per_req = [max(1, -(-L // page_size)) for L in seq_lens]
+    num_pages = sum(pages_per_req) + spare_pages
+    kc = randn_bf16((num_pages, page_size, Hkv, ATTN_DIM), g)
+    vc = randn_bf16((num_pages, page_size, Hkv, ATTN_DIM), g)
+    perm = torch.randperm(num_pages, generator=g).to(torch.int32)
+    table = torch.full((R, max(pages_per_req)), -1, dtype=torch.int32)
+    at = 0
+    for r, n in enumerate(pages_per_req):
+        table[r, :n] = perm[at:at + n]
+        at += n
+    T = sum(qlens)
+    q = randn_bf16((T, Hq, ATTN_DIM), g)
+    blocks = torch.full((T, k), -1, dtype=torch.int32)
+    t = 0
+    for r in range(R):
+        for i in range(qlens[r]):
+            pos = seq_lens[r] - qlens[r] + i
+            vis = max(0, min((pos + 1) // TOKENS_PER_KEY, seq_lens[r] // TOKENS_PER_KEY))
+            n = min(k, vis)
+            if n:
+                pick = torch.randperm(vis, generator=g)[:n].sort().values.to(torch.int32)
+                blocks[t, :n] = pick
+            t += 1
+    cu = [0]
+    for n in qlens:
+        cu.append(cu[-1] + n)
+    return AttentionInputs(name=name, q=q, k_cache=kc, v_cache=vc, page_table=table,
+                           cu_seqlens_q=torch.tensor(cu, dtype=torch.int32),
+                           seq_lens=torch.tensor(seq_lens, dtype=torch.int32), blocks=blocks,
+                           meta={"seed": seed, "context_tokens": list(seq_lens), "query_rows": list(qlens),
+                                 "heads": (Hq, Hkv), "page_size": page_size, "k": k})

@@ -452,6 +452,112 @@ class AttentionBench:
                                 scale=1.0 / 16.0, threads=threads)
 
 
+class MixedBench:
+    """A mixed decode + prefill batch from the paged cache in one
+    qsa_mqa_paged_batch call (decode kernel, metadata kernel, prefill kernel,
+    fix-up: four launches chained with programmatic dependent launches)."""
+    kernel = "prefill_kernel"
+    bound = "hbm+tensor"
+    unit = "us"
+
+    def __init__(self, cfg: int, dev: torch.device, seed: int):
+        import sparse_attention_block_qsa_b200 as qsa
+        self.qsa = qsa
+        self.inp = b = wl.make_config(cfg, seed=seed)
+        self.name = b.name
+        self.dev = dev
+        D, Q = b.num_decodes, b.decode_query_len
+        sl = b.seq_lens.tolist()
+        cu = b.cu_seqlens_q.tolist()
+        self.dec_bytes, self.pre_flops = self.accounting(b)
+        ws = qsa.paged_batch_workspace_size(len(sl), D, Q, b.T, b.W)
+        per_copy = b.q.numel() * 2 + b.k_cache.numel() * 2 + b.T * b.W * 4
+        self.copies = max(2, math.ceil(2 * L2_BYTES / per_copy))
+        self.bufs = [(b.q.to(dev), b.k_cache.to(dev), b.page_table.to(dev), b.cu_seqlens_q.to(dev),
+                      b.seq_lens.to(dev), torch.empty((b.T, b.W), dtype=torch.float32, device=dev),
+                      torch.empty(ws // 4 + 4, dtype=torch.float32, device=dev)) for _ in range(self.copies)]
+        self.units = 1.0
+        self.launches_per_step = 4
+        self.h2d = (b.q.numel() + b.k_cache.numel()) * 2 + (b.page_table.numel() + len(sl) + len(cu)) * 4
+        self.d2h = b.T * b.W * 4
+        self.dtype = "bf16"
+        self.config = {"workload": b.name, "decode_requests": D, "decode_query_len": Q,
+                       "prefill_rows": b.T - D * Q, "context_tokens": sl, "page_size": b.page_size, "W": b.W,
+                       "decode_bytes": self.dec_bytes, "prefill_flop": self.pre_flops, "input_copies": self.copies,
+                       "l2": f"steps rotate over {self.copies} input copies "
+                             f"({self.copies * per_copy / 2**20:.0f} MiB > 2x L2)"}
+
+    @staticmethod
+    def accounting(b):
+        """Decode bytes of the decode requests (the vLLM PR's formula) and
+        prefill FLOPs of the prefill rows (2 * 4 * 128 per visible key, the
+        row at position p seeing min((p + 1) // 4, L // 4) keys)."""
+        D, Q = b.num_decodes, b.decode_query_len
+        sl = b.seq_lens.tolist()
+        cu = b.cu_seqlens_q.tolist()
+        vis = 0
+        for r in range(D, len(sl)):
+            qlen = cu[r + 1] - cu[r]
+            for i in range(qlen):
+                pos = sl[r] - qlen + i
+                vis += max(0, min((pos + 1) // 4, sl[r] // 4, b.W))
+        return decode_bytes(sl[:D], Q), 2 * 4 * 128 * vis
+
+    def _launch(self, q, kc, pt, cu, sl, out, ws):
+        b = self.inp
+        self.qsa.mqa_paged_batch(q, kc, pt, cu, sl, b.num_decodes, b.decode_query_len, b.W, out=out, workspace=ws)
+
+    def step(self, i: int):
+        self._launch(*self.bufs[i % self.copies])
+
+    def throughput(self, seconds_per_step: float) -> float:
+        return seconds_per_step * 1e6
+
+    def roofline(self, seconds_per_step: float, peaks: dict) -> dict:
+        """The step against the sum of its parts' roofline times: the decode
+        bytes at the HBM copy bandwidth, plus the prefill rows' bound, the
+        larger of their FLOPs at the bf16 peak and their fp32 score rows
+        (W columns each) at the HBM bandwidth."""
+        b = self.inp
+        pre_rows = b.T - b.num_decodes * b.decode_query_len
+        pre = max(self.pre_flops / (peaks["bf16_tflops"] * 1e12), pre_rows * b.W * 4 / (peaks["hbm_gbs"] * 1e9))
+        ideal = self.dec_bytes / (peaks["hbm_gbs"] * 1e9) + pre
+        return {"bound": self.bound, "ideal_us": ideal * 1e6, "achieved_us": seconds_per_step * 1e6,
+                "frac": ideal / seconds_per_step, "unit": "us", "traffic": None,
+                "peak": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]},
+                "peak_source": peaks["source"]}
+
+    def e2e_setup(self):
+        b = self.inp
+        self.host = [t.pin_memory() for t in (b.q, b.k_cache, b.page_table, b.cu_seqlens_q, b.seq_lens)]
+        self.host_out = torch.empty((b.T, b.W), dtype=torch.float32).pin_memory()
+
+    def e2e_step(self, i: int):
+        bufs = self.bufs[i % self.copies]
+        for dst, src in zip(bufs[:5], self.host):
+            dst.copy_(src, non_blocking=True)
+        self._launch(*bufs)
+        self.host_out.copy_(bufs[5], non_blocking=True)
+
+    def oracle_sample(self):
+        b = self.inp
+        return 64 / b.T, "the 16 decode rows and 48 prefill rows, every column (scaled to the full batch by rows)"
+
+    def oracle_step(self, threads: int = 0):
+        import oracle
+        b = self.inp
+        D, Q = b.num_decodes, b.decode_query_len
+        oracle.decode(b.q[:D * Q].reshape(D, Q, 4, 128), b.k_cache, b.page_table[:D], b.seq_lens[:D], b.W,
+                      threads=threads)
+        r = D
+        first = int(b.cu_seqlens_q[r])
+        n = int(b.cu_seqlens_q[r + 1]) - first
+        rows = b.q[first + n - 48:first + n].reshape(1, 48, 4, 128)
+        # the last 48 rows of the prefill request: a request cut to those rows
+        cut = b.seq_lens[r:r + 1].clone()
+        oracle.decode(rows, b.k_cache, b.page_table[r:r + 1], cut, b.W, threads=threads)
+
+
 def make_bench(cfg: int, dev, seed: int, fp8: bool = False):
     if fp8 and cfg not in (1, 2, 3):
         raise ValueError("the fp8 key cache applies to the decode configurations 1-3")
@@ -459,6 +565,8 @@ def make_bench(cfg: int, dev, seed: int, fp8: bool = False):
         return DecodeBench(cfg, dev, seed, fp8)
     if cfg == 6:
         return AttentionBench(cfg, dev, seed)
+    if cfg == 7:
+        return MixedBench(cfg, dev, seed)
     return PrefillBench(cfg, dev, seed)
 
 
@@ -570,7 +678,7 @@ def cpu_baseline(b, budget_s: float = 10.0) -> dict:
 # ------------------------------------------------------------------ main
 
 HEADLINE = 3            # the long-context spec-decode workload: the decode roofline target
-ALL_CONFIGS = [3, 1, 2, 4, 5, 6]
+ALL_CONFIGS = [3, 1, 2, 4, 5, 6, 7]
 
 
 def run_reference(args, rank: int, world: int):
@@ -591,7 +699,7 @@ def run_reference(args, rank: int, world: int):
     value = inp_bench.throughput(per_step)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": inp_bench.unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "higher_is_better": inp_bench.unit != "us", "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": inp_bench.config,
             "cpu_baseline": {"value": value, "unit": inp_bench.unit, "cores": threads, "kind": "oracle",
                              "sample": f"{what}; fp64 C oracle on {threads} host threads"},
@@ -607,7 +715,10 @@ class _HostOnly:
         self.inp = wl.make_config(cfg)
         self.fp8 = fp8 and cfg in (1, 2, 3)
         self.k_scale = 1.0
-        if cfg == 6:
+        if cfg == 7:
+            self.unit = "us"
+            self.config = {"workload": self.inp.name, "W": self.inp.W}
+        elif cfg == 6:
             a = self.inp
             self.units, _, _ = AttentionBench._accounting(a, a.q.shape[1], a.k_cache.shape[2])
             self.unit = "GB/s"
@@ -630,9 +741,13 @@ class _HostOnly:
             self.config = {"workload": p.name, "keys": p.Nk, "W": p.W}
 
     def throughput(self, s):
+        if self.unit == "us":
+            return s * 1e6
         return self.units / s / (1e9 if self.unit == "GB/s" else 1e12)
 
     def oracle_sample(self):
+        if self.cfg == 7:
+            return MixedBench.oracle_sample(self)
         if self.cfg == 6:
             return AttentionBench.oracle_sample(self)
         if self.cfg in (1, 2, 3):
@@ -640,7 +755,9 @@ class _HostOnly:
         return 64 / self.inp.T, "64 query rows of the batch, every column (scaled to the full batch)"
 
     def oracle_step(self, threads):
-        if self.cfg == 6:
+        if self.cfg == 7:
+            MixedBench.oracle_step(self, threads)
+        elif self.cfg == 6:
             AttentionBench.oracle_step(self, threads)
         elif self.cfg in (1, 2, 3):
             DecodeBench.oracle_step(self, threads)
@@ -683,26 +800,33 @@ def measure(cfg: int, args, world: int, rank: int, local: int, cpu_budget_s: flo
     rec = None
     if rank == 0:
         peaks = read_peaks()
-        value = b.throughput(per_step) * world
-        if b.bound == "hbm":
+        value = b.throughput(per_step) * (world if b.unit != "us" else 1)
+        if hasattr(b, "roofline"):
+            pass
+        elif b.bound == "hbm":
             achieved = b.units / kernel_s / 1e9
             peak, unit = peaks["hbm_gbs"], "GB/s"
         else:
             achieved = b.units / kernel_s / 1e12
             peak, unit = peaks["bf16_tflops"], "TFLOP/s"
-        roofline = {"bound": b.bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                    "traffic": read_traffic(b.kernel, b.name), "kernel": b.kernel,
-                    "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst figure)"
-                    if peaks["source"] == "measured" else "fallback"}
+        if hasattr(b, "roofline"):
+            roofline = b.roofline(kernel_s, peaks)
+        else:
+            roofline = {"bound": b.bound, "achieved": achieved, "peak": peak, "unit": unit,
+                        "frac": achieved / peak, "traffic": read_traffic(b.kernel, b.name), "kernel": b.kernel,
+                        "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst figure)"
+                        if peaks["source"] == "measured" else "fallback"}
         pub = None if args.kv_fp8 else PUBLISHED.get(cfg)
         conf = dict(b.config)
         if pub:
             conf["published_reference"] = pub[2]
         rec = {"workload": b.name, "value": value, "unit": b.unit, "ms_per_step": per_step * 1e3,
+               "higher_is_better": b.unit != "us",
                "us_per_step": per_step * 1e6,
                "vs_baseline": (value / pub[1]) if pub and pub[0] == b.unit else None,
                "dtype": getattr(b, "dtype", "bf16"), "config": conf, "roofline": roofline,
-               "e2e": {"value": b.throughput(e2e_s) * world, "unit": b.unit, "h2d_bytes_per_step": b.h2d,
+               "e2e": {"value": b.throughput(e2e_s) * (world if b.unit != "us" else 1), "unit": b.unit,
+                       "h2d_bytes_per_step": b.h2d,
                        "d2h_bytes_per_step": b.d2h, "ms_per_step": e2e_s * 1e3},
                "gpu_launches": args.steps * b.launches_per_step, "clocks": clocks, "device_error": dev_err}
         rec.update(extra)
@@ -748,7 +872,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=None, choices=[1, 2, 3, 4, 5, 6],
+    ap.add_argument("--config", type=int, default=None, choices=[1, 2, 3, 4, 5, 6, 7],
                     help="one workload only (default: all five, the long-context spec-decode one as the headline)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

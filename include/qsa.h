@@ -353,6 +353,52 @@ qsa_status_t qsa_sparse_attention(const void* q, int64_t q_stride_t, int64_t q_s
 
 size_t qsa_sparse_attention_workspace_size(int64_t T, int32_t Hq, int32_t Hkv, int32_t width);
 
+/*
+ * qsa_mqa_paged_batch - indexer scores of a mixed decode + prefill batch,
+ * every request read from the paged compressed key cache, in one call.
+ *
+ * The vLLM PR "Separate prefill and decode paths for QSA indexer" ("Main
+ * changes") splits a batch into uniform decode requests and prefill
+ * requests, computes the visible block counts in the metadata step (vLLM
+ * qsa_cache.py, the metadata kernel: logical positions and visible_blocks,
+ * chained to its consumers with programmatic dependent launches) and scores
+ * each part with its own kernel.  This call does the same on the device, on
+ * `stream`, in four launches chained the same way: the decode kernel on
+ * requests 0 .. D-1; a metadata kernel that gives every prefill row its key
+ * interval and packs the prefill requests' keys out of their pages; the
+ * tcgen05 prefill kernel on those rows; a fix-up that sets the scores of keys
+ * whose page is missing to -inf.
+ *
+ *   q          bf16 [T, 4, 128] (row stride q_stride_t, head stride
+ *              q_stride_h; multiples of 8; 16-byte aligned): the D *
+ *              decode_query_len decode rows first, then the prefill rows.
+ *   k_cache..  as qsa_mqa_decode (page_size 8 .. 1024), for all R requests.
+ *   cu_seqlens_q int32 [R + 1], seq_lens int32 [R] (tokens, query rows
+ *              included): the caller guarantees cu_seqlens_q[r] =
+ *              r * decode_query_len for r <= D (the device contents are not
+ *              read on the host).  Row i of request r sits at logical
+ *              position seq_lens[r] - qlen_r + i.
+ *   num_decodes D requests (0 .. R) are decodes with decode_query_len
+ *              (1 .. 4) rows each; R - D <= 8192 prefill requests with
+ *              (R - D) * W <= 2^31 - 1.
+ *   out        fp32 [T, W], row stride out_stride: out[t, n] = score of
+ *              request-local key n for n < visible(t) (and n < W), -inf
+ *              otherwise; keys in missing pages are -inf.
+ *   workspace  16-byte aligned, qsa_mqa_paged_batch_workspace_size(R, D,
+ *              decode_query_len, T, W) bytes (packed keys and intervals);
+ *              smaller returns QSA_ERR_WORKSPACE.  Not needed (may be NULL)
+ *              when every request is a decode.
+ */
+qsa_status_t qsa_mqa_paged_batch(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k_cache,
+                                 int64_t num_pages, int32_t page_size, int64_t k_page_stride, int64_t k_row_stride,
+                                 const int32_t* page_table, int64_t pt_stride, int32_t max_pages,
+                                 const int32_t* cu_seqlens_q, const int32_t* seq_lens, int32_t R, int32_t num_decodes,
+                                 int32_t decode_query_len, int64_t T, float scale, float* out, int64_t out_stride,
+                                 int32_t W, void* workspace, size_t workspace_bytes, void* stream);
+
+size_t qsa_mqa_paged_batch_workspace_size(int32_t R, int32_t num_decodes, int32_t decode_query_len, int64_t T,
+                                          int32_t W);
+
 #ifdef __cplusplus
 }
 #endif

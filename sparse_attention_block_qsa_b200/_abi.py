@@ -46,6 +46,9 @@ SIGNATURES = {
                                        _vp, _i64, _i32, _vp, _vp, _i32, _vp, _i64, _i32, _i64, _vp, _f32,
                                        _vp, _i64, _vp, _vp, _sz, _vp]),
     "qsa_sparse_attention_workspace_size": (_sz, [_i64, _i32, _i32, _i32]),
+    "qsa_mqa_paged_batch": (C.c_int, [_vp, _i64, _i64, _vp, _i64, _i32, _i64, _i64, _vp, _i64, _i32, _vp, _vp,
+                                      _i32, _i32, _i32, _i64, _f32, _vp, _i64, _i32, _vp, _sz, _vp]),
+    "qsa_mqa_paged_batch_workspace_size": (_sz, [_i32, _i32, _i32, _i64, _i32]),
 }
 
 STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_ALIGNMENT", 3: "QSA_ERR_UNSUPPORTED",
@@ -366,3 +369,42 @@ def sparse_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
         token_idx.stride(0), width, T, _ptr(gate), float(scale), _ptr(out), out.stride(0), _ptr(lse),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, lse
+
+
+def paged_batch_workspace_size(R: int, num_decodes: int, decode_query_len: int, T: int, W: int) -> int:
+    return int(lib().qsa_mqa_paged_batch_workspace_size(R, num_decodes, decode_query_len, T, W))
+
+
+def mqa_paged_batch(q: torch.Tensor, k_cache: torch.Tensor, page_table: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                    seq_lens: torch.Tensor, num_decodes: int, decode_query_len: int, W: int, scale: float = SCALE,
+                    out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """Scores of a mixed batch from the paged cache: q bf16 [T, 4, 128] (the
+    num_decodes x decode_query_len decode rows first), k_cache bf16 [pages,
+    page_size, 1, 128], page_table int32 [R, max_pages], cu_seqlens_q int32
+    [R + 1], seq_lens int32 [R] -> out fp32 [T, W] (request-local key
+    columns).  The workspace is allocated here by torch when not given."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(page_table, "page_table", torch.int32, 2)
+    _index_checks(cu_seqlens_q, seq_lens)
+    if q.shape[1:] != (4, 128) or q.stride(2) != 1:
+        raise ValueError("q must be [T, 4, 128] with unit feature stride")
+    if k_cache.shape[2:] != (1, 128) or k_cache.stride(3) != 1 or page_table.stride(1) != 1:
+        raise ValueError("k_cache must be [pages, page_size, 1, 128]; page_table needs a unit column stride")
+    T = q.shape[0]
+    R = seq_lens.shape[0]
+    if out is None:
+        out = torch.empty((T, W), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, 2)
+    if out.shape != (T, W) or out.stride(1) != 1:
+        raise ValueError("out must be [T, W] with unit column stride")
+    if workspace is None:
+        need = paged_batch_workspace_size(R, num_decodes, decode_query_len, T, W)
+        workspace = torch.empty(max(need, 16) // 4 + 4, dtype=torch.float32, device=q.device)
+    _check("qsa_mqa_paged_batch", lib().qsa_mqa_paged_batch(
+        _ptr(q), q.stride(0), q.stride(1), _ptr(k_cache), k_cache.shape[0], k_cache.shape[1], k_cache.stride(0),
+        k_cache.stride(1), _ptr(page_table), page_table.stride(0), page_table.shape[1], _ptr(cu_seqlens_q),
+        _ptr(seq_lens), R, num_decodes, decode_query_len, T, scale, _ptr(out), out.stride(0), W,
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out

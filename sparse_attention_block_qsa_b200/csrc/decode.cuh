@@ -233,6 +233,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   const int gw = blockIdx.x * WARPS + warp;
   const int nw = gridDim.x * WARPS;
 
+  // Launched as a programmatic dependent (the mixed-batch path): wait for the
+  // previous kernel's writes, then let the next kernel begin launching.  A
+  // no-op for an ordinary launch.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
   // ---- the lengths load goes out first.  With at most 32 requests every
   // warp builds the request plan in its own registers (lane b: request b), so
   // no warp waits for another; otherwise one block-wide scan in shared memory.

@@ -192,6 +192,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   if (warp == 1) tmem_alloc(&S.tmem_base, TMEM_COLS);
 
+  // Launched as a programmatic dependent (the mixed-batch path): wait for the
+  // previous kernel's writes (ks, ke and the keys may come from it), then let
+  // the next kernel begin launching.  A no-op for an ordinary launch.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
   // ---- plan: key-tile range of every token tile.  16 threads share a token
   // tile, 4 rows each; every load of a pass is issued before any is used, so
   // a pass costs one memory round trip.

@@ -17,6 +17,7 @@
 #include "prefill.cuh"
 #include "topk.cuh"
 #include "attention.cuh"
+#include "paged_batch.cuh"
 
 namespace {
 
@@ -157,6 +158,24 @@ qsa_status_t launch_status(const char* what) {
   return ok();
 }
 
+// Launch with programmatic stream serialization (the kernel may begin
+// launching while the previous kernel on the stream finishes; every kernel of
+// this library waits with griddepcontrol.wait before its first global read).
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---------------------------------------------------------------- intervals
 __global__ void prefill_intervals_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ seq_lens,
                                          const int32_t* __restrict__ key_offsets, int32_t S, int64_t T,
@@ -224,7 +243,7 @@ qsa_status_t validate_prefill(const PrefillArgs& a) {
   return QSA_OK;
 }
 
-qsa_status_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
+qsa_status_t launch_prefill(const PrefillArgs& a, cudaStream_t stream, bool pdl = false) {
   int sms = 0;
   qsa_status_t st = device_info(&sms);
   if (st != QSA_OK) return st;
@@ -259,7 +278,10 @@ qsa_status_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     CUtensorMap tm_out;
     memset(&tm_out, 0, sizeof tm_out);
     p.store_map = encode_f32_store_map(&tm_out, p.out, a.W, p.T, a.out_stride) ? 1 : 0;
-    if (a.f16)
+    if (pdl)
+      launch_pdl(a.f16 ? qsa::prefill::prefill_kernel<true> : qsa::prefill::prefill_kernel<false>, dim3(sms),
+                 dim3(qsa::prefill::NUM_THREADS), qsa::prefill::SMEM_BYTES, stream, tm_q, tm_k, tm_out, p);
+    else if (a.f16)
       qsa::prefill::prefill_kernel<true><<<sms, qsa::prefill::NUM_THREADS, qsa::prefill::SMEM_BYTES, stream>>>(
           tm_q, tm_k, tm_out, p);
     else
@@ -413,8 +435,12 @@ qsa_status_t qsa_selftest_bounded_wait(uint64_t timeout_ns, int32_t arrive, void
 // and are scaled by k_scale; bf16 and fp16 keys take 2 (k_scale == 1).
 extern "C++" {
 template <qsa::decode::Fmt F, bool GEN>
-static void launch_decode(int sms, const qsa::decode::Params& p, cudaStream_t stream) {
-  qsa::decode::decode_kernel<F, GEN><<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES, stream>>>(p);
+static void launch_decode(int sms, const qsa::decode::Params& p, cudaStream_t stream, bool pdl) {
+  if (pdl)
+    launch_pdl(qsa::decode::decode_kernel<F, GEN>, dim3(sms), dim3(qsa::decode::NUM_THREADS), qsa::decode::SMEM_BYTES,
+               stream, p);
+  else
+    qsa::decode::decode_kernel<F, GEN><<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES, stream>>>(p);
 }
 }
 
@@ -424,7 +450,7 @@ static qsa_status_t decode_common(const void* q, int64_t q_stride_b, int64_t q_s
                                   int64_t k_page_stride, int64_t k_row_stride, const int32_t* page_table,
                                   int64_t pt_stride, int32_t max_pages, const int32_t* seq_lens, int32_t B, int32_t Q,
                                   float scale, float* out, int64_t out_stride_b, int64_t out_stride_t, int32_t W,
-                                  void* stream) {
+                                  void* stream, bool pdl = false) {
   if (B < 0 || W < 0) return fail(QSA_ERR_INVALID_ARG, "B and W must be non-negative");
   if (Q < 1 || Q > 4) return fail(QSA_ERR_UNSUPPORTED, "Q = %d query tokens per request; 1..4 supported", Q);
   if (page_size < 8 || page_size > 1024)
@@ -516,9 +542,12 @@ static qsa_status_t decode_common(const void* q, int64_t q_stride_b, int64_t q_s
     p.out = out + (int64_t)b0 * out_stride_b;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     using qsa::decode::Fmt;
-    if (fmt == Fmt::E4M3) pow2 ? launch_decode<Fmt::E4M3, false>(sms, p, s) : launch_decode<Fmt::E4M3, true>(sms, p, s);
-    else if (fmt == Fmt::F16) pow2 ? launch_decode<Fmt::F16, false>(sms, p, s) : launch_decode<Fmt::F16, true>(sms, p, s);
-    else pow2 ? launch_decode<Fmt::BF16, false>(sms, p, s) : launch_decode<Fmt::BF16, true>(sms, p, s);
+    if (fmt == Fmt::E4M3)
+      pow2 ? launch_decode<Fmt::E4M3, false>(sms, p, s, pdl) : launch_decode<Fmt::E4M3, true>(sms, p, s, pdl);
+    else if (fmt == Fmt::F16)
+      pow2 ? launch_decode<Fmt::F16, false>(sms, p, s, pdl) : launch_decode<Fmt::F16, true>(sms, p, s, pdl);
+    else
+      pow2 ? launch_decode<Fmt::BF16, false>(sms, p, s, pdl) : launch_decode<Fmt::BF16, true>(sms, p, s, pdl);
     st = launch_status("decode kernel");
     if (st != QSA_OK) return st;
   }
@@ -837,6 +866,127 @@ qsa_status_t qsa_sparse_attention(const void* q, int64_t q_stride_t, int64_t q_s
   const int64_t warps = T * Hq;
   qsa::attn::combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(p);
   return launch_status("sparse attention combine kernel");
+}
+
+// Workspace of qsa_mqa_paged_batch: the prefill keys packed (at most W per
+// prefill request, 256 bytes each), then ks and ke of the prefill rows.
+static size_t paged_batch_layout(int32_t R, int32_t D, int64_t prefill_rows, int32_t W, size_t* ks_off,
+                                 size_t* ke_off) {
+  const size_t keys = (size_t)(R - D) * (size_t)W * 256;
+  const size_t iv = ((size_t)prefill_rows * 4 + 15) & ~size_t(15);
+  *ks_off = keys;
+  *ke_off = keys + iv;
+  return keys + 2 * iv;
+}
+
+size_t qsa_mqa_paged_batch_workspace_size(int32_t R, int32_t num_decodes, int32_t decode_query_len, int64_t T,
+                                          int32_t W) {
+  if (R <= 0 || num_decodes < 0 || num_decodes > R || W <= 0 || T < 0) return 0;
+  const int64_t rows = T - (int64_t)num_decodes * (num_decodes > 0 ? decode_query_len : 0);
+  if (rows <= 0 || num_decodes == R) return 0;
+  size_t a, b;
+  return paged_batch_layout(R, num_decodes, rows, W, &a, &b);
+}
+
+qsa_status_t qsa_mqa_paged_batch(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k_cache,
+                                 int64_t num_pages, int32_t page_size, int64_t k_page_stride, int64_t k_row_stride,
+                                 const int32_t* page_table, int64_t pt_stride, int32_t max_pages,
+                                 const int32_t* cu_seqlens_q, const int32_t* seq_lens, int32_t R, int32_t num_decodes,
+                                 int32_t decode_query_len, int64_t T, float scale, float* out, int64_t out_stride,
+                                 int32_t W, void* workspace, size_t workspace_bytes, void* stream) {
+  const int32_t D = num_decodes;
+  if (R < 0 || D < 0 || D > R || T < 0 || W < 0) return fail(QSA_ERR_INVALID_ARG, "negative or inconsistent counts");
+  if (D > 0 && (decode_query_len < 1 || decode_query_len > 4))
+    return fail(QSA_ERR_UNSUPPORTED, "decode_query_len = %d; 1..4 supported", decode_query_len);
+  const int64_t row0 = (int64_t)D * (D > 0 ? decode_query_len : 0);
+  if (row0 > T) return fail(QSA_ERR_INVALID_ARG, "T = %lld rows is below the decode rows %lld", (long long)T,
+                            (long long)row0);
+  if (T > row0 && D == R) return fail(QSA_ERR_INVALID_ARG, "rows past the decode requests need prefill requests");
+  if (R - D > qsa::batch::MAX_PREFILL)
+    return fail(QSA_ERR_UNSUPPORTED, "%d prefill requests; at most %d per call", R - D, qsa::batch::MAX_PREFILL);
+  if ((int64_t)(R - D) * W > INT32_MAX)
+    return fail(QSA_ERR_UNSUPPORTED, "prefill requests x W = %lld keys exceeds 2^31 - 1", (long long)(R - D) * W);
+  if (page_size < 8 || page_size > 1024)
+    return fail(QSA_ERR_UNSUPPORTED, "page_size = %d; supported page sizes are 8 .. 1024", page_size);
+  if (T == 0 || W == 0) return ok();
+  if (!q || !k_cache || !cu_seqlens_q || !seq_lens || !out || (max_pages > 0 && !page_table))
+    return fail(QSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(cu_seqlens_q, 4) || !aligned(seq_lens, 4)) return fail(QSA_ERR_ALIGNMENT, "index arrays must be 4-byte aligned");
+  if (T > 1 && out_stride < W) return fail(QSA_ERR_INVALID_ARG, "out_stride below W");
+  if (T > 1 && (q_stride_t <= 0 || q_stride_t % 8 != 0))
+    return fail(QSA_ERR_ALIGNMENT, "q_stride_t must be a positive multiple of 8");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t ostride = T > 1 ? out_stride : W;
+  const int64_t qst = T > 1 ? q_stride_t : 4 * q_stride_h;
+  qsa_status_t st;
+  // every check that can fail runs before the first launch
+  qsa::batch::Params bp;
+  PrefillArgs pa{};
+  const bool has_prefill = T > row0;
+  if (has_prefill) {
+    size_t ks_off = 0, ke_off = 0;
+    const size_t need = paged_batch_layout(R, D, T - row0, W, &ks_off, &ke_off);
+    if (!workspace || workspace_bytes < need)
+      return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes; %zu needed", workspace_bytes, need);
+    if (!aligned(workspace, 16)) return fail(QSA_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+    if (num_pages < 1 || num_pages > INT32_MAX) return fail(QSA_ERR_INVALID_ARG, "num_pages out of range");
+    if (!aligned(k_cache, 16) || k_row_stride < 128 || k_row_stride % 8 != 0 ||
+        (num_pages > 1 && (k_page_stride <= 0 || k_page_stride % 8 != 0)))
+      return fail(QSA_ERR_ALIGNMENT, "k_cache must be 16-byte aligned with strides that are multiples of 8");
+    if (max_pages > 0 && R > 1 && pt_stride < max_pages)
+      return fail(QSA_ERR_INVALID_ARG, "pt_stride = %lld is below max_pages = %d", (long long)pt_stride, max_pages);
+    char* ws = static_cast<char*>(workspace);
+    bp.cu = cu_seqlens_q;
+    bp.seq_lens = seq_lens;
+    bp.R = R;
+    bp.D = D;
+    bp.row0 = row0;
+    bp.T = T;
+    bp.k_cache = static_cast<const uint16_t*>(k_cache);
+    bp.num_pages = num_pages;
+    bp.page_size = page_size;
+    bp.k_page_stride = num_pages > 1 ? k_page_stride : 0;
+    bp.k_row_stride = k_row_stride;
+    bp.page_table = page_table;
+    bp.pt_stride = pt_stride;
+    bp.max_pages = max_pages;
+    bp.W = W;
+    bp.packed = reinterpret_cast<uint16_t*>(ws);
+    bp.ks = reinterpret_cast<int32_t*>(ws + ks_off);
+    bp.ke = reinterpret_cast<int32_t*>(ws + ke_off);
+    bp.out = out;
+    bp.out_stride = ostride;
+    const int64_t cap = (int64_t)(R - D) * W;
+    pa = PrefillArgs{static_cast<const uint16_t*>(q) + row0 * qst, qst, q_stride_h, bp.packed, 128, cap,
+                     bp.ks, bp.ke, T - row0, scale, out + row0 * ostride, ostride, W};
+    st = validate_prefill(pa);
+    if (st != QSA_OK) return st;
+    const Range rw = span(workspace, 1, 1, 0, 1, 0, 1, 0, (int64_t)need);
+    if (overlaps(rw, span(out, 4, T, ostride, 1, 0, 1, 0, W)) || overlaps(rw, span(q, 2, T, qst, 4, q_stride_h, 1, 0, 128)))
+      return fail(QSA_ERR_INVALID_ARG, "workspace overlaps q or out");
+  }
+  // 1. decode rows: requests 0 .. D-1, decode_query_len rows each (validated, then launched)
+  if (D > 0) {
+    const int32_t Q = decode_query_len;
+    st = decode_common(q, Q * qst, qst, q_stride_h, k_cache, qsa::decode::Fmt::BF16, 1.f, num_pages, page_size,
+                       k_page_stride, k_row_stride, page_table, pt_stride, max_pages, seq_lens, D, Q, scale, out,
+                       Q * ostride, ostride, W, stream, /*pdl=*/true);
+    if (st != QSA_OK) return st;
+  }
+  if (!has_prefill) return ok();
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != QSA_OK) return st;
+  // 2. the metadata step for the prefill requests: intervals and packed keys
+  launch_pdl(qsa::batch::gather_kernel, dim3(sms * 4), dim3(qsa::batch::THREADS), qsa::batch::SMEM_BYTES, s, bp);
+  st = launch_status("paged-batch metadata kernel");
+  if (st != QSA_OK) return st;
+  // 3. prefill rows over the packed keys
+  st = launch_prefill(pa, s, /*pdl=*/true);
+  if (st != QSA_OK) return st;
+  // 4. keys whose page is missing
+  launch_pdl(qsa::batch::fixup_kernel, dim3(R - D), dim3(qsa::batch::THREADS), 0, s, bp);
+  return launch_status("paged-batch fix-up kernel");
 }
 
 }  // extern "C"

@@ -194,8 +194,11 @@ def pin_prefill_intervals_follow_cache_writer(orc):
 
 def pin_decode_exact_bruteforce(orc):
     rng = np.random.default_rng(1)
+    # query lengths past 4 are the prefill rows of a request read from the
+    # paged cache (a mixed decode + prefill batch scores them the same way)
     cases = [(1, 1, 8, [37]), (3, 4, 8, [70, 41, 2]), (2, 2, 16, [130, 75]),
-             (3, 3, 8, [0, 66, 19]), (2, 4, 16, [64, 3])]
+             (3, 3, 8, [0, 66, 19]), (2, 4, 16, [64, 3]), (2, 9, 16, [70, 41]), (1, 33, 8, [200]),
+             (1, 12, 8, [5])]
     for B, Q, ps, lens in cases:
         q, kc, table, sl, W = paged_case(rng, B, Q, ps, lens)
         got = orc.decode(q, kc, table, sl, W, scale=1.0, threads=2)

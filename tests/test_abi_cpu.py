@@ -257,3 +257,26 @@ def test_expand_rejects(kw, code):
     st = L.qsa_expand_block_indices(a["blk"], a["bs"], a["k"], a["cu"], a["sl"], a["R"], a["T"], a["tok"], a["tks"],
                                     None)
     assert st == code, L.qsa_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=5), INVALID), (dict(R=-1), INVALID), (dict(Qd=5), UNSUP), (dict(Qd=0), UNSUP),
+    (dict(T=3), INVALID), (dict(D=4, T=20), INVALID), (dict(ps=7), UNSUP), (dict(W=1 << 30), UNSUP),
+    (dict(q=0), INVALID), (dict(ost=10), INVALID), (dict(wsb=100), WS), (dict(ws=A + 7 * S + 8), ALIGN),
+])
+def test_paged_batch_rejects(kw, code):
+    a = dict(q=A, qst=512, qsh=128, k=A + S, pages=100, ps=64, kps=64 * 128, krs=128, pt=A + 2 * S, pts=10, maxp=10,
+             cu=A + 3 * S, sl=A + 3 * S + 4096, R=4, D=2, Qd=4, T=40, scale=0.088, out=A + 4 * S, ost=1000, W=1000,
+             ws=A + 7 * S, wsb=1 << 30)
+    a.update(kw)
+    L = qsa.lib()
+    st = L.qsa_mqa_paged_batch(a["q"], a["qst"], a["qsh"], a["k"], a["pages"], a["ps"], a["kps"], a["krs"], a["pt"],
+                               a["pts"], a["maxp"], a["cu"], a["sl"], a["R"], a["D"], a["Qd"], a["T"], a["scale"],
+                               a["out"], a["ost"], a["W"], a["ws"], a["wsb"], None)
+    assert st == code, L.qsa_last_error_detail().decode()
+
+
+def test_paged_batch_workspace_size():
+    # 2 prefill requests x W = 1000 keys x 256 bytes, then ks and ke of the 32 prefill rows
+    assert qsa.paged_batch_workspace_size(4, 2, 4, 40, 1000) == 2 * 1000 * 256 + 2 * 128
+    assert qsa.paged_batch_workspace_size(4, 4, 4, 16, 1000) == 0       # decodes only

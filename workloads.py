@@ -207,6 +207,7 @@ CONFIG_NAMES = {
     4: "prefill_t8192_prefix50144",
     5: "prefill_4x4096_prefix102400_top512",
     6: "core_attention_b16_q4_top512_h24x2_d256_ps64",
+    7: "mixed_batch_16decode_plus_prefill2048_after30000_ps64",
 }
 TOPK_K = 512
 
@@ -254,6 +255,11 @@ def make_config(idx: int, seed: int = 0):
         # 24 query heads over 2 KV heads of dimension 256, 64-token pages
         ctx = lognormal_contexts(16, 3508, 102400, 16 * 51200, seed)
         return make_attention(name, ctx, [4] * 16, 24, 2, 64, TOPK_K, seed=seed)
+    if idx == 7:
+        # workload 2's 16 decode requests and one prefill request of 2,048 new
+        # rows after 30,000 cached tokens, one paged pool (64-row pages)
+        ctx = lognormal_contexts(16, 1536, 43876, 16 * 10240, seed)
+        return make_paged_batch(name, ctx, 1, [2048], [30000], 64, seed=seed)
     raise KeyError(idx)
 
 
@@ -320,3 +326,58 @@ def make_attention(name: str, seq_lens: list[int], qlens: list[int], Hq: int, Hk
                            seq_lens=torch.tensor(seq_lens, dtype=torch.int32), blocks=blocks,
                            meta={"seed": seed, "context_tokens": list(seq_lens), "query_rows": list(qlens),
                                  "heads": (Hq, Hkv), "page_size": page_size, "k": k})
+
+
+@dataclass
+class PagedBatchInputs:
+    """A mixed batch read from the paged compressed key cache (all tensors on
+    the CPU): D decode requests with Q query rows each, then prefill requests
+    with their own numbers of new rows; q packed in that order."""
+    name: str
+    q: torch.Tensor            # bf16 [T, 4, 128]
+    k_cache: torch.Tensor      # bf16 [num_pages, page_size, 1, 128]
+    page_table: torch.Tensor   # int32 [R, max_pages]
+    cu_seqlens_q: torch.Tensor # int32 [R + 1]
+    seq_lens: torch.Tensor     # int32 [R]
+    num_decodes: int
+    decode_query_len: int
+    page_size: int
+    W: int
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def T(self) -> int:
+        return self.q.shape[0]
+
+
+def make_paged_batch(name: str, decode_lens: list[int], Q: int, prefill_new: list[int],
+                     prefill_prefix: list[int], page_size: int, seed: int, W: int | None = None) -> PagedBatchInputs:
+    """Decode requests of the given context lengths (query rows included)
+    followed by prefill requests with `prefill_new` rows after
+    `prefill_prefix` cached tokens; one paged pool for all of them (pages
+    handed out by a random permutation, one spare, -1 past a request's
+    pages), N(0, 1) bf16 queries and keys."""
+    g = _gen(seed)
+    lens = list(decode_lens) + [p + n for p, n in zip(prefill_prefix, prefill_new)]
+    qlens = [Q] * len(decode_lens) + list(prefill_new)
+    tokens_per_page = TOKENS_PER_KEY * page_size
+    pages_per_req = [max(1, -(-L // tokens_per_page)) for L in lens]
+    num_pages = sum(pages_per_req) + 1
+    k_cache = randn_bf16((num_pages, page_size, 1, DIM), g)
+    perm = torch.randperm(num_pages, generator=g).to(torch.int32)
+    table = torch.full((len(lens), max(pages_per_req)), -1, dtype=torch.int32)
+    at = 0
+    for r, n in enumerate(pages_per_req):
+        table[r, :n] = perm[at:at + n]
+        at += n
+    q = randn_bf16((sum(qlens), HEADS, DIM), g)
+    cu = [0]
+    for n in qlens:
+        cu.append(cu[-1] + n)
+    if W is None:
+        W = max(lens) // TOKENS_PER_KEY
+    return PagedBatchInputs(name=name, q=q, k_cache=k_cache, page_table=table,
+                            cu_seqlens_q=torch.tensor(cu, dtype=torch.int32),
+                            seq_lens=torch.tensor(lens, dtype=torch.int32), num_decodes=len(decode_lens),
+                            decode_query_len=Q, page_size=page_size, W=W,
+                            meta={"seed": seed, "context_tokens": lens, "query_rows": qlens})

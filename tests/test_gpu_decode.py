@@ -12,6 +12,7 @@ pytestmark = pytest.mark.gpu
 
 qsa = pytest.importorskip("sparse_attention_block_qsa_b200")
 SCALE = 1.0 / np.sqrt(128.0)
+DEV = torch.device("cuda")
 
 
 def run_case(d: wl.DecodeInputs, q=None, k_cache=None, out=None, W=None):
@@ -241,3 +242,36 @@ def test_decode_many_requests(B, Q, ps):
 
 def test_decode_fp8_many_requests():
     run_case_fp8(_many(1500, 4, 16, seed=99))
+
+
+# ---------------------------------------------------------------- large pages, dense and padded rows
+
+@pytest.mark.parametrize("ps", [32, 64, 128, 1024])
+@pytest.mark.parametrize("Q", [1, 4])
+def test_decode_large_pages_and_masks(ps, Q):
+    lens = [1, 4, 129, 8 * ps + 5, 3000, 20000, 4 * ps * 3]
+    d = wl.make_decode("bulk", lens, Q=Q, page_size=ps, seed=ps + Q, table_pad=1, W=max(lens) // 4 - 100)
+    t = d.page_table.clone()
+    t[4, 1] = -1                                   # a missing page
+    t[5, 2] = d.k_cache.shape[0] + 9               # a page outside the pool
+    d.page_table = t
+    run_case(d)
+
+
+@pytest.mark.parametrize("B", [1, 17, 32])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_decode_dense_and_padded_rows_agree(B, dtype):
+    """The same keys in dense rows and in rows padded to 136 elements give
+    bitwise the same scores (the row stride only moves the loads)."""
+    lens = torch.randint(1, 12000, (B,), generator=torch.Generator().manual_seed(B)).tolist()
+    d = wl.make_decode("dense_vs_padded", lens, Q=3, page_size=64, seed=B)
+    q, kc = d.q.to(dtype).to(DEV), d.k_cache.to(dtype).to(DEV)
+    padded = torch.zeros(kc.shape[0], kc.shape[1], 1, 136, dtype=dtype, device=DEV)
+    padded[..., :128] = kc
+    pt, sl = d.page_table.to(DEV), d.seq_lens.to(DEV)
+    dense = qsa.mqa_decode(q, kc, pt, sl, d.W)
+    regs = qsa.mqa_decode(q, padded[..., :128], pt, sl, d.W)
+    torch.cuda.synchronize()
+    assert qsa.device_error() == 0
+    assert torch.equal(torch.isneginf(dense), torch.isneginf(regs))
+    assert torch.equal(dense, regs)

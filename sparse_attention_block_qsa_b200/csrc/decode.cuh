@@ -48,7 +48,6 @@
 #pragma once
 
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 
 #include "sm100.cuh"
 
@@ -126,10 +125,15 @@ __device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, uint3
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Two E4M3 codes (low byte = lower feature) -> fp16x2, exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Four E4M3 codes (byte i = feature i) -> two fp16x2 words (features 0, 1
+// and 2, 3), exact: one hardware conversion per pair.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t four, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(four));
 }
 
 // bf16x2 word -> fp16x2 word of the two values times dn (a power of two).
@@ -501,7 +505,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
           if constexpr (FP8) {
             // words 2s, 2s + 1 = bytes 0-3 (s even) or 4-7 (s odd) of chunk s / 2
             const uint32_t four = (s & 1) ? kv8[u0 + v][s >> 1].y : kv8[u0 + v][s >> 1].x;
-            mma_f16_16816(d[v], qa[s], e4m3x2_to_f16x2(four), e4m3x2_to_f16x2(four >> 16));
+            uint32_t b0, b1;
+            e4m3x4_to_f16x2x2(four, b0, b1);
+            mma_f16_16816(d[v], qa[s], b0, b1);
           } else if constexpr (F == Fmt::F16) {
             const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[u0 + v]);
             mma_f16_16816(d[v], qa[s], w[2 * s], w[2 * s + 1]);

@@ -231,27 +231,41 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(const Params p) {
 
   // Warp w gathers token slots n = w + 4i (i < 8) of every chunk, one K row
   // and one V row per slot (32 lanes x 16 bytes each).  Their row offsets
-  // are found four chunks at a time: lane l resolves slot w + 4 (l & 7) of
-  // chunk 4 win + (l >> 3) (list entry, then page entry: two dependent loads
-  // per four chunks instead of per chunk) and the loads shuffle them out.
-  int64_t win_off = -1;  // this lane's resolved element offset of KV head g, or -1: masked
-  auto resolve = [&](int win) {
+  // are found four chunks (a window) at a time: lane l resolves slot
+  // w + 4 (l & 7) of chunk 4 win + (l >> 3), list entry first, then page
+  // entry, and the loads shuffle them out.  The two dependent loads of a
+  // window run a window ahead: its list entries are loaded when the previous
+  // window starts and its page entries two chunks later, so no chunk waits
+  // on them.
+  auto tok_of = [&](int win) -> int {
     const int c = 4 * win + (lane >> 3);
     const int e = e_begin + c * CHUNK + warp + WARPS * (lane & 7);
-    const int j = e < e_end ? __ldg(tok_row + e) : -1;
-    int64_t off = -1;
-    if (j >= 0 && j <= pos && j < L) {
-      const int lp = j / p.page_size;
-      const int page = lp < p.max_pages ? __ldg(pt_row + lp) : -1;
-      if (page >= 0 && (int64_t)page < p.num_pages)
-        off = (int64_t)page * p.kv_page_stride + (int64_t)(j - lp * p.page_size) * p.kv_row_stride +
-              (int64_t)g * p.kv_head_stride;
-    }
-    win_off = off;
+    return e < e_end ? __ldg(tok_row + e) : -1;
   };
+  auto page_of = [&](int j) -> int {
+    if (j < 0 || j > pos || j >= L) return -1;
+    const int lp = j / p.page_size;
+    return lp < p.max_pages ? __ldg(pt_row + lp) : -1;
+  };
+  auto offset_of = [&](int j, int page) -> int64_t {
+    if (j < 0 || j > pos || j >= L || page < 0 || (int64_t)page >= p.num_pages) return -1;
+    const int lp = j / p.page_size;
+    return (int64_t)page * p.kv_page_stride + (int64_t)(j - lp * p.page_size) * p.kv_row_stride +
+           (int64_t)g * p.kv_head_stride;
+  };
+  int64_t win_off = -1;                          // this window's offsets (-1: masked)
+  int tok_nx = tok_of(0), page_nx = -1;          // the next window's entries as they arrive
+  page_nx = page_of(tok_nx);
+  win_off = offset_of(tok_nx, page_nx);
+  tok_nx = tok_of(1);
   // Gather chunk c into stage s (chunks are loaded in order 0, 1, 2, ...).
   auto load_chunk = [&](int c, int s) {
-    if ((c & 3) == 0) resolve(c >> 2);
+    if ((c & 3) == 0 && c > 0) {                 // window c / 4 begins: its pages were looked up
+      win_off = offset_of(tok_nx, page_nx);
+      tok_nx = tok_of((c >> 2) + 1);
+    } else if ((c & 3) == 2) {
+      page_nx = page_of(tok_nx);                 // page entries of the next window
+    }
     const uint32_t kbase = smem_addr(kv_s + (2 * s) * KV_STAGE_BYTES);
     const uint32_t vbase = smem_addr(kv_s + (2 * s + 1) * KV_STAGE_BYTES);
     const int u = lane;

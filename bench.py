@@ -83,14 +83,26 @@ def read_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def source_hash() -> str:
-    """Digest of the kernel sources (every file of csrc/) with comments and
-    blank space removed, so that it changes exactly when the code does."""
+# The device sources of each timed kernel (its own header and the shared
+# sm_100a helpers).
+KERNEL_SOURCES = {
+    "decode_kernel": ["decode.cuh", "sm100.cuh"],
+    "prefill_kernel": ["prefill.cuh", "sm100.cuh"],
+    "topk_stream_kernel": ["topk.cuh", "sm100.cuh"],
+    "attn_kernel": ["attention.cuh", "sm100.cuh"],
+}
+
+
+def source_hash(kernel: str | None = None) -> str:
+    """Digest of a kernel's device sources (every file of csrc/ when kernel is
+    None) with comments and blank space removed, so that it changes exactly
+    when that code does."""
     import hashlib
     import re
     src = os.path.join(ROOT, "sparse_attention_block_qsa_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(src)):
+    files = KERNEL_SOURCES.get(kernel) if kernel else None
+    for f in sorted(files or os.listdir(src)):
         with open(os.path.join(src, f), encoding="utf-8") as fh:
             text = fh.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -106,7 +118,7 @@ def read_traffic(kernel: str, workload: str):
     path = os.path.join(ROOT, "profiles", "dram_traffic.md")
     if not os.path.exists(path):
         return None
-    sha = source_hash()
+    sha = source_hash(kernel)
     for line in open(path):
         parts = [p.strip() for p in line.strip().strip("|").split("|")]
         if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload and parts[2] == sha:

@@ -104,6 +104,8 @@ __device__ __forceinline__ void row_request(const int32_t* __restrict__ cu, cons
 
 // ---------------------------------------------------------------- expansion
 
+constexpr int EXPAND_MAX_K = 512;   // block-hint width limit (QSA docs, "Core Attention")
+
 struct ExpandParams {
   const int32_t* blk;   // [T, k]
   int64_t blk_stride;
@@ -125,10 +127,17 @@ __global__ void __launch_bounds__(256) expand_kernel(const ExpandParams p) {
   const int32_t* src = p.blk + t * p.blk_stride;
   int32_t* dst = p.tok + t * p.tok_stride;
   const int width = 4 * p.k + 3;
+  // every block entry of the row (k <= 512: 16 per lane) in one round trip
+  int bv[EXPAND_MAX_K / 32];
+#pragma unroll
+  for (int u = 0; u < EXPAND_MAX_K / 32; ++u) {
+    const int i = u * 32 + lane;
+    bv[u] = i < p.k ? __ldg(src + i) : -1;
+  }
   int n = 0;  // tokens written so far (warp-uniform)
-  for (int i0 = 0; i0 < p.k; i0 += 32) {
-    const int i = i0 + lane;
-    const int b = i < p.k ? __ldg(src + i) : -1;
+#pragma unroll
+  for (int u = 0; u < EXPAND_MAX_K / 32; ++u) {
+    const int b = bv[u];
     const unsigned keep = __ballot_sync(0xffffffffu, b >= 0);
     if (b >= 0) {
       const int at = n + 4 * __popc(keep & ((1u << lane) - 1u));

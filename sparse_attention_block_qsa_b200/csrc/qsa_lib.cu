@@ -676,8 +676,19 @@ qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_s
   float* ws = static_cast<float*>(workspace);
   PrefillArgs pa{q, q_stride_t, q_stride_h, k, k_stride, Nk, ks, ke, T, scale, ws, (int64_t)W, W};
   TopkArgs ta{ws, (int64_t)W, nullptr, T, W, topk_k, idx, idx_stride};
-  qsa_status_t st = validate_topk(ta);
-  if (st != QSA_OK) return st;
+  {
+    // k, W and alignment; the workspace holds one chunk of rows, not T, so
+    // its overlaps are checked below against the chunk actually used
+    TopkArgs one = ta;
+    one.rows = std::min<int64_t>(T, 1);
+    one.idx_stride = topk_k;
+    qsa_status_t st = validate_topk(one);
+    if (st != QSA_OK) return st;
+  }
+  if (T > INT32_MAX) return fail(QSA_ERR_UNSUPPORTED, "rows = %lld exceeds 2^31 - 1", (long long)T);
+  if (T > 1 && idx_stride < topk_k)
+    return fail(QSA_ERR_INVALID_ARG, "idx_stride = %lld is below k = %d", (long long)idx_stride, topk_k);
+  qsa_status_t st;
   if (T < 0 || Nk < 0) return fail(QSA_ERR_INVALID_ARG, "T and Nk must be non-negative");
   if (T == 0) return ok();
   if (!workspace) return fail(QSA_ERR_WORKSPACE, "workspace is null");

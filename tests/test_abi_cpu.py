@@ -280,3 +280,19 @@ def test_paged_batch_workspace_size():
     # 2 prefill requests x W = 1000 keys x 256 bytes, then ks and ke of the 32 prefill rows
     assert qsa.paged_batch_workspace_size(4, 2, 4, 40, 1000) == 2 * 1000 * 256 + 2 * 128
     assert qsa.paged_batch_workspace_size(4, 4, 4, 16, 1000) == 0       # decodes only
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="passes validation and would launch on fake addresses")
+def test_fused_workspace_is_checked_per_chunk_not_per_batch():
+    """A small workspace followed in memory by idx (within T x W floats of the
+    workspace start) is valid: the workspace only ever holds one chunk of rows.
+    Validation passes and the call fails later, at the first CUDA call (no GPU
+    here)."""
+    L = qsa.lib()
+    T, W, kk = 4096, 26624, 512
+    ws_bytes = 64 << 20
+    ws = A + 5 * S
+    idx = ws + ws_bytes + 4096                       # right after the workspace
+    st = L.qsa_mqa_prefill_topk(A, 512, 128, A + S, 128, 106496, A + 2 * S, A + 3 * S, T, 0.088, W, kk, idx, kk,
+                                ws, ws_bytes, None)
+    assert st == 5, L.qsa_last_error_detail().decode()   # QSA_ERR_CUDA: validation passed

@@ -14,7 +14,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqsa.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("qsa_lib.cu",)]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "decode.cuh", "prefill.cuh", "topk.cuh")] + [
+DEPS = SOURCES + sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
     os.path.join(INCLUDE, "qsa.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

@@ -88,7 +88,7 @@ def read_peaks() -> dict:
 KERNEL_SOURCES = {
     "decode_kernel": ["decode.cuh", "sm100.cuh"],
     "prefill_kernel": ["prefill.cuh", "sm100.cuh"],
-    "topk_stream_kernel": ["topk.cuh", "sm100.cuh"],
+    "topk_pipe_kernel": ["topk.cuh", "sm100.cuh"],
     "attn_kernel": ["attention.cuh", "sm100.cuh"],
 }
 
@@ -820,7 +820,7 @@ def measure(cfg: int, args, world: int, rank: int, local: int, cpu_budget_s: flo
             "prefill_us": pre * 1e6, "topk_us": top * 1e6,
             "topk": {"bound": "hbm", "achieved": topk_bytes / top / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": topk_bytes / top / 1e9 / peaks["hbm_gbs"], "bytes_per_step": topk_bytes,
-                     "traffic": read_traffic("topk_stream_kernel", b.name)}}
+                     "traffic": read_traffic("topk_pipe_kernel", b.name)}}
         fused = b.time_fused()
         if fused is not None:
             extra["fused_l2_workspace"] = fused

@@ -140,7 +140,7 @@ qsa_status_t device_info(int* sms) {
         {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel<true>), qsa::prefill::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::attn::attn_kernel), qsa::attn::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_rows_kernel), qsa::topk::ROWS_SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::topk::topk_stream_kernel), qsa::topk::STREAM_SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::topk::topk_pipe_kernel), qsa::topk::PIPE_SMEM_BYTES},
     };
     for (auto& k : kernels) {
       e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k.bytes);
@@ -348,9 +348,8 @@ qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream, float* pred_sta
   const int64_t max_grid = pred_state ? kPredFloats : INT32_MAX;
   if (p.vec4 && a.W % 4 == 0) {
     // rows start on 16-byte boundaries: stream them with bulk copies
-    const int64_t grid = std::min<int64_t>(std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::STREAM_CTAS_PER_SM), max_grid);
-    qsa::topk::topk_stream_kernel<<<(unsigned)grid, qsa::topk::STREAM_THREADS, qsa::topk::STREAM_SMEM_BYTES,
-                                    stream>>>(p);
+    const int64_t grid = std::min<int64_t>(std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::PIPE_CTAS_PER_SM), max_grid);
+    qsa::topk::topk_pipe_kernel<<<(unsigned)grid, qsa::topk::PIPE_THREADS, qsa::topk::PIPE_SMEM_BYTES, stream>>>(p);
   } else {
     const int64_t grid = std::min<int64_t>(std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::ROWS_CTAS_PER_SM), max_grid);
     qsa::topk::topk_rows_kernel<<<(unsigned)grid, qsa::topk::THREADS, qsa::topk::ROWS_SMEM_BYTES, stream>>>(p);

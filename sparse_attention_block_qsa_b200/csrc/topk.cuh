@@ -4,13 +4,10 @@
 //
 // Persistent CTAs, each over a contiguous range of rows (neighbouring query
 // rows score alike).  Two kernels share the selection logic:
-//  * topk_stream_kernel (rows 16-byte aligned, W a multiple of 4), three
-//    CTAs per SM: a producer warp streams every row of the CTA's range as
-//    16 KB bulk copies into a 2-slot shared-memory ring without pausing
-//    between rows; 8 selecting warps read the ring.  The selection work is
-//    latency-bound (short phases between barriers), so the SM holds as many
-//    CTAs as registers allow (72 per thread) and while one CTA resolves a
-//    row the others keep streaming.
+//  * topk_pipe_kernel (rows 16-byte aligned, W a multiple of 4), two CTAs per
+//    SM: a producer warp streams the rows as 16 KB bulk copies, filtering
+//    warps build each row's candidate list while selecting warps resolve the
+//    previous row (described beside the kernel).
 //  * topk_rows_kernel (any alignment): 8 warps read each row with batched
 //    loads themselves.
 // Per row:
@@ -43,7 +40,6 @@ namespace topk {
 constexpr int THREADS = 256;          // selecting threads (both kernels)
 constexpr int NWARPS = THREADS / 32;
 constexpr int ROWS_CTAS_PER_SM = 4;
-constexpr int STREAM_CTAS_PER_SM = 3;
 constexpr int HBITS = 11;
 constexpr int HBINS = 1 << HBITS;
 constexpr int HSHIFT = 32 - HBITS;
@@ -56,8 +52,6 @@ constexpr int FBINS = 2048;           // fast-path histogram
 constexpr uint32_t ZERO_KEY = 0x80000000u;
 constexpr float PREDICT_MARGIN = 0.9f;
 constexpr int CHUNK = 4096;           // floats per ring slot (16 KB)
-constexpr int NST = 2;                // ring slots
-constexpr int STREAM_THREADS = THREADS + 32;
 static_assert(FBINS == HBINS, "the fast path and the exact path share one histogram");
 
 struct Params {
@@ -338,10 +332,11 @@ __device__ __forceinline__ void find_bin(Sel& S, uint32_t k) {
 }
 
 // Fast-path resolution on the candidate list (all keys >= key_lo, at least
-// k of them, S.hist zeroed): marks the selected columns.
+// k of them, S.hist zeroed): marks the selected columns.  With kth != nullptr
+// the k-th largest key is returned there too.
 template <class Sync>
 __device__ __forceinline__ void resolve_candidates(const Params& p, Sel& S, uint32_t key_lo, uint32_t& thr,
-                                                   uint32_t& need_tie) {
+                                                   uint32_t& need_tie, uint32_t* kth = nullptr) {
   const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t k = (uint32_t)p.k;
   const uint32_t kmax = S.kmax;
@@ -377,6 +372,11 @@ __device__ __forceinline__ void resolve_candidates(const Params& p, Sel& S, uint
         rank += (ko > key) || (ko == key && jo < j);
       }
       if (have && rank < needB) atomicOr(&S.gt[j >> 5], 1u << (j & 31));
+      if (kth != nullptr && have && rank == needB - 1) S.lo = key;
+    }
+    if (kth != nullptr) {
+      Sync::sync();
+      *kth = S.lo;
     }
     thr = 0;
     need_tie = 0;
@@ -390,6 +390,7 @@ __device__ __forceinline__ void resolve_candidates(const Params& p, Sel& S, uint
   });
   thr = lo;
   need_tie = nd;
+  if (kth != nullptr) *kth = lo;
 }
 
 // Exact threshold among the list keys of the boundary bin: histogram levels
@@ -616,39 +617,91 @@ __global__ void __launch_bounds__(THREADS, ROWS_CTAS_PER_SM) topk_rows_kernel(co
   if (p.pred_state && tid == 0) p.pred_state[blockIdx.x] = pred;
 }
 
-// -------------------------------------------------------------- streaming kernel
+constexpr size_t ROWS_SMEM_BYTES = sizeof(Sel);
 
-struct StreamSmem {
-  float ring[NST * CHUNK];
-  uint64_t full[NST];
-  uint64_t empty[NST];
+// -------------------------------------------------------------- pipelined kernel
+//
+// topk_pipe_kernel (rows 16-byte aligned, W a multiple of 4), two CTAs per
+// SM.  Resolving a row (short phases between barriers) takes about as long as
+// streaming it (measured: ~13k cycles each per row at W = 26,624), so when
+// the same warps do both, the copies stall while a row resolves.  Here the
+// roles are split so the two overlap:
+//  * a producer warp streams the CTA's rows as 16 KB bulk copies into a
+//    3-slot ring, without pausing between rows;
+//  * 8 filtering warps compare every score with the prediction and append
+//    candidates to a staging list (warp w owns list segment w; positions
+//    from a warp scan of the lanes' counts);
+//  * 8 selecting warps (threads 0..255, the helpers above) take the staged
+//    list of row r (copying it frees the staging list for row r+1) and
+//    resolve it while the filtering warps already read row r+1.
+// A row whose list misses (fewer than k candidates, or a full segment) is
+// filtered once more from L2 by the selecting warps with the threshold moved
+// toward its k-th value (x 0.85 below, x 1.08 above the prediction), and only
+// if that misses too goes to the exact path; rows without a prediction take
+// the exact path.  The prediction used for row r+1 is the one known when its
+// filtering starts (a miss refreshes it, as in the rows kernel).
+
+constexpr int PIPE_SEL_WARPS = NWARPS;   // threads 0 .. 255
+constexpr int PIPE_FILT_WARPS = 8;
+constexpr int PIPE_FILT_THREADS = PIPE_FILT_WARPS * 32;
+constexpr int PIPE_SEGS = NWARPS / PIPE_FILT_WARPS;      // list segments per filtering warp
+constexpr int PIPE_WARP_CAP = PIPE_SEGS * SEG;
+constexpr int PIPE_THREADS = (PIPE_SEL_WARPS + PIPE_FILT_WARPS + 1) * 32;
+constexpr int PIPE_CTAS_PER_SM = 2;
+constexpr int PNST = 3;                  // ring slots
+constexpr uint32_t FILTER_BAR = 2;       // named barrier of the filtering warps
+constexpr float REFILTER_DOWN = 0.85f;
+constexpr float REFILTER_UP = 1.08f;
+static_assert(PIPE_SEGS * PIPE_FILT_WARPS == NWARPS, "the filtering warps own every list segment");
+
+struct PipeList {   // one row's candidates as the filtering warps leave them
+  uint32_t key[CAP];
+  int32_t idx[CAP];
+  uint32_t cnt[PIPE_FILT_WARPS];  // entries appended by each filtering warp (may pass PIPE_WARP_CAP)
+  uint32_t kmax;
+  float pred;                     // the threshold the row was filtered with (0: none)
+  int stop;
+};
+
+struct PipeSmem {
+  float ring[PNST * CHUNK];
+  uint64_t full[PNST];
+  uint64_t empty[PNST];
+  uint64_t list_full;
+  uint64_t list_empty;
+  float pred_next;                // the latest prediction (written by the selecting warps)
+  PipeList F;
   Sel sel;
 };
 
-constexpr size_t STREAM_SMEM_BYTES = sizeof(StreamSmem) + 128;
-constexpr size_t ROWS_SMEM_BYTES = sizeof(Sel);
+constexpr size_t PIPE_SMEM_BYTES = sizeof(PipeSmem) + 128;
+static_assert(PIPE_CTAS_PER_SM * (PIPE_SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs fit an SM's shared memory");
 
-__global__ void __launch_bounds__(STREAM_THREADS, STREAM_CTAS_PER_SM) topk_stream_kernel(const Params p) {
+__global__ void __launch_bounds__(PIPE_THREADS, PIPE_CTAS_PER_SM) topk_pipe_kernel(const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  StreamSmem& M = *reinterpret_cast<StreamSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  PipeSmem& M = *reinterpret_cast<PipeSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   Sel& S = M.sel;
+  PipeList& F = M.F;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t k = (uint32_t)p.k;
   const int64_t r_begin = (int64_t)blockIdx.x * p.rows / gridDim.x;
   const int64_t r_end = (int64_t)(blockIdx.x + 1) * p.rows / gridDim.x;
 
   if (tid == 0) {
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < PNST; ++s) {
       mbar_init(&M.full[s], 1);
-      mbar_init(&M.empty[s], NWARPS);
+      mbar_init(&M.empty[s], PIPE_FILT_WARPS);
     }
+    mbar_init(&M.list_full, 1);
+    mbar_init(&M.list_empty, 1);
+    M.pred_next = p.pred_state ? p.pred_state[blockIdx.x] : 0.f;
     S.abort = 0;
     fence_mbar_init();
   }
-  for (int i = tid; i < BM_WORDS; i += STREAM_THREADS) S.gt[i] = S.tie[i] = 0;
+  for (int i = tid; i < BM_WORDS; i += PIPE_THREADS) S.gt[i] = S.tie[i] = 0;
   __syncthreads();
 
-  if (warp == NWARPS) {
+  if (warp == PIPE_SEL_WARPS + PIPE_FILT_WARPS) {
     // ================= producer: every chunk of every row, back to back
     if (lane == 0) {
       uint32_t it = 0;
@@ -656,8 +709,8 @@ __global__ void __launch_bounds__(STREAM_THREADS, STREAM_CTAS_PER_SM) topk_strea
         const int len4 = (row_len(p, r) + 3) & ~3;  // within the row: W is a multiple of 4
         const float* row = p.scores + r * p.stride;
         for (int c0 = 0; c0 < len4; c0 += CHUNK, ++it) {
-          const int s = it % NST;
-          if (!mbar_wait(&M.empty[s], ((it / NST) & 1) ^ 1, &S.abort)) {
+          const int s = it % PNST;
+          if (!mbar_wait(&M.empty[s], ((it / PNST) & 1) ^ 1, &S.abort)) {
             if (atomicExch(&S.abort, 1) == 0) record_device_error(QSA_DEVERR_WAIT_TIMEOUT);
             break;
           }
@@ -671,62 +724,58 @@ __global__ void __launch_bounds__(STREAM_THREADS, STREAM_CTAS_PER_SM) topk_strea
         }
       }
       // the last copy into every slot must land before the block may retire
-      for (uint32_t i = it > (uint32_t)NST ? it - NST : 0u; i < it; ++i)
-        if (!mbar_wait(&M.full[i % NST], (i / NST) & 1, nullptr)) break;
+      for (uint32_t i = it > (uint32_t)PNST ? it - PNST : 0u; i < it; ++i)
+        if (!mbar_wait(&M.full[i % PNST], (i / PNST) & 1, nullptr)) break;
     }
     __syncwarp();
-    return;  // the selecting threads never wait for this warp
+    return;
   }
 
-  // ================= 8 selecting warps
-  float pred = p.pred_state ? p.pred_state[blockIdx.x] : 0.f;
-  uint32_t it = 0;
-  for (int64_t r = r_begin; r < r_end; ++r) {
-    const float* row = p.scores + r * p.stride;
-    const int len = row_len(p, r);
-    const int len4 = (len + 3) & ~3;
-    const bool fast = pred > 0.f;
-    start_row(S);
-    ConsumerSync::sync();
-    uint32_t kmax = 0, cnt = 0, zc = 0;
-    uint32_t count = 0;  // this warp's list entries (warp-uniform)
-    for (int c0 = 0; c0 < len4; c0 += CHUNK, ++it) {
-      const int s = it % NST;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&M.full[s], (it / NST) & 1, &S.abort));
-      if (ok) {
-        const float4* ring4 = reinterpret_cast<const float4*>(M.ring + s * CHUNK);
-        const bool tail = c0 + CHUNK > len;
-        uint32_t mask = 0;  // fast path: bit 4u + e = score e of this lane's u-th float4 is a candidate
+  if (warp >= PIPE_SEL_WARPS) {
+    // ================= filtering warps
+    const int fw = warp - PIPE_SEL_WARPS, ftid = tid - PIPE_SEL_WARPS * 32;
+    uint32_t it = 0;
+    for (int64_t r = r_begin; r < r_end; ++r) {
+      const uint32_t i_row = (uint32_t)(r - r_begin);
+      if (ftid == 0) {
+        // the staging list is free once the selecting warps copied the previous row
+        if (!mbar_wait(&M.list_empty, (i_row & 1) ^ 1, &S.abort) && atomicExch(&S.abort, 1) == 0)
+          record_device_error(QSA_DEVERR_WAIT_TIMEOUT);
+        F.pred = *(volatile float*)&M.pred_next;
+        F.kmax = 0;
+        F.stop = *(volatile int*)&S.abort;
+      }
+      named_barrier_sync(FILTER_BAR, PIPE_FILT_THREADS);
+      if (F.stop) break;
+      const float pred = F.pred;
+      const bool fast = pred > 0.f;
+      const int len = row_len(p, r);
+      const int len4 = (len + 3) & ~3;
+      uint32_t kmax = 0, count = 0;  // count: this warp's list entries (warp-uniform)
+      for (int c0 = 0; c0 < len4; c0 += CHUNK, ++it) {
+        const int s = it % PNST;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&M.full[s], (it / PNST) & 1, &S.abort));
+        if (!ok) {
+          if (lane == 0 && atomicExch(&S.abort, 1) == 0) record_device_error(QSA_DEVERR_WAIT_TIMEOUT);
+        } else if (fast) {
+          const float4* ring4 = reinterpret_cast<const float4*>(M.ring + s * CHUNK);
+          const bool tail = c0 + CHUNK > len;
+          constexpr int U = CHUNK / 4 / PIPE_FILT_THREADS;  // float4 per thread per chunk
+          uint32_t mask = 0;  // bit 4u + e: score e of this lane's u-th float4 is a candidate
 #pragma unroll
-        for (int u = 0; u < CHUNK / 4 / THREADS; ++u) {
-          const int f = u * THREADS + tid;
-          float4 x = ring4[f];
-          const int j0 = c0 + 4 * f;
-          if (tail) {
-            if (j0 >= len) x.x = -INFINITY;
-            if (j0 + 1 >= len) x.y = -INFINITY;
-            if (j0 + 2 >= len) x.z = -INFINITY;
-            if (j0 + 3 >= len) x.w = -INFINITY;
-          }
-          if (fast) {
+          for (int u = 0; u < U; ++u) {
+            const int f = u * PIPE_FILT_THREADS + ftid;
+            float4 x = ring4[f];
+            const int j0 = c0 + 4 * f;
+            if (tail) {
+              if (j0 >= len) x.x = -INFINITY;
+              if (j0 + 1 >= len) x.y = -INFINITY;
+              if (j0 + 2 >= len) x.z = -INFINITY;
+              if (j0 + 3 >= len) x.w = -INFINITY;
+            }
             mask |= (uint32_t)(x.x >= pred) << (4 * u) | (uint32_t)(x.y >= pred) << (4 * u + 1) |
                     (uint32_t)(x.z >= pred) << (4 * u + 2) | (uint32_t)(x.w >= pred) << (4 * u + 3);
-          } else {
-            const float xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t key = score_key(xs[e]);
-              if (key) {
-                ++cnt;
-                if (key == ZERO_KEY) ++zc;
-                else atomicAdd(&S.hist[key >> HSHIFT], 1u);
-              }
-            }
           }
-        }
-        if (fast) {
-          // positions from a warp scan of the lanes' candidate counts; then
-          // each lane copies its few candidates from the ring into the list
           const uint32_t nl = __popc(mask);
           uint32_t incl = nl;
 #pragma unroll
@@ -739,57 +788,105 @@ __global__ void __launch_bounds__(STREAM_THREADS, STREAM_CTAS_PER_SM) topk_strea
           while (mask) {
             const int b = __ffs(mask) - 1;
             mask &= mask - 1;
-            const int f = (b >> 2) * THREADS + tid;
+            const int f = (b >> 2) * PIPE_FILT_THREADS + ftid;
             const float x = M.ring[s * CHUNK + 4 * f + (b & 3)];
             const uint32_t key = __float_as_uint(x) | 0x80000000u;  // x >= pred > 0
-            if (pos < SEG) {
-              S.cand_key[warp * SEG + pos] = key;
-              S.cand_idx[warp * SEG + pos] = c0 + 4 * f + (b & 3);
+            if (pos < (uint32_t)PIPE_WARP_CAP) {
+              F.key[fw * PIPE_WARP_CAP + pos] = key;
+              F.idx[fw * PIPE_WARP_CAP + pos] = c0 + 4 * f + (b & 3);
             }
             kmax = max(kmax, key);
             ++pos;
           }
         }
-      } else if (lane == 0 && atomicExch(&S.abort, 1) == 0) {
-        record_device_error(QSA_DEVERR_WAIT_TIMEOUT);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&M.empty[s]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&M.empty[s]);
-    }
-    uint32_t thr = 0, need_tie = 0;
-    bool done = false;
-    if (fast) {
       kmax = __reduce_max_sync(0xffffffffu, kmax);
       if (lane == 0) {
-        atomicMax(&S.kmax, kmax);
-        S.seg_cnt[warp] = count;
+        atomicMax(&F.kmax, kmax);
+        F.cnt[fw] = count;
       }
-      ConsumerSync::sync();
-      bool overflow;
-      if (list_size(S, overflow) >= k && !overflow) {
-        resolve_candidates<ConsumerSync>(p, S, __float_as_uint(pred) | 0x80000000u, thr, need_tie);
-        done = true;
-      }
-      ConsumerSync::sync();
-      if (!done) exact_select<ConsumerSync>(p, S, row, len, false, thr, need_tie);
-    } else {
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      zc = __reduce_add_sync(0xffffffffu, zc);
-      if (lane == 0) {
-        atomicAdd(&S.total, cnt);
-        if (zc) atomicAdd(&S.zeros, zc);
-      }
-      ConsumerSync::sync();
-      exact_select<ConsumerSync>(p, S, row, len, true, thr, need_tie);
+      named_barrier_sync(FILTER_BAR, PIPE_FILT_THREADS);
+      if (ftid == 0) mbar_arrive(&M.list_full);
+    }
+    return;
+  }
+
+  // ================= 8 selecting warps
+  for (int64_t r = r_begin; r < r_end; ++r) {
+    const uint32_t i_row = (uint32_t)(r - r_begin);
+    const float* row = p.scores + r * p.stride;
+    const int len = row_len(p, r);
+    start_row(S);
+    if (tid == 0) {
+      if (!mbar_wait(&M.list_full, i_row & 1, &S.abort) && atomicExch(&S.abort, 1) == 0)
+        record_device_error(QSA_DEVERR_WAIT_TIMEOUT);
+      S.stop = *(volatile int*)&S.abort;
     }
     ConsumerSync::sync();
-    if (!done) pred = next_prediction(thr);  // a miss refreshes the prediction
-    write_row<ConsumerSync>(p, S, p.idx + r * p.idx_stride, (len + 31) >> 5, need_tie);
-    if (tid == 0) S.stop = *(volatile int*)&S.abort;  // one reading for every warp
-    ConsumerSync::sync();
     if (S.stop) break;
+    // take the staged list: segment 2w + h of filtering warp w holds its
+    // entries h * SEG .. h * SEG + SEG - 1
+    const float pred = F.pred;
+    uint32_t n = 0;
+    bool overflow = false;
+#pragma unroll
+    for (int w = 0; w < PIPE_FILT_WARPS; ++w) {
+      n += F.cnt[w];
+      overflow |= F.cnt[w] > (uint32_t)PIPE_WARP_CAP;
+    }
+    const bool hit = pred > 0.f && n >= k && !overflow;
+    if (hit) {
+      for (int i = tid; i < CAP; i += THREADS) {
+        const uint32_t c = F.cnt[i / PIPE_WARP_CAP], slot = (uint32_t)(i % PIPE_WARP_CAP);
+        if (slot < c) {
+          S.cand_key[i] = F.key[i];
+          S.cand_idx[i] = F.idx[i];
+        }
+      }
+      if (tid < NWARPS) {
+        const uint32_t c = F.cnt[tid / PIPE_SEGS];
+        const uint32_t first = (uint32_t)(tid % PIPE_SEGS) * SEG;
+        S.seg_cnt[tid] = c > first ? min(c - first, (uint32_t)SEG) : 0u;
+      }
+      if (tid == 0) S.kmax = F.kmax;
+    }
+    ConsumerSync::sync();
+    if (tid == 0) mbar_arrive(&M.list_empty);  // the filtering warps may stage the next row
+
+    uint32_t thr = 0, need_tie = 0, kth = 0;
+    bool done = false, refreshed = false;
+    if (hit) {
+      resolve_candidates<ConsumerSync>(p, S, __float_as_uint(pred) | 0x80000000u, thr, need_tie);
+      done = true;
+    } else if (pred > 0.f) {
+      // filter the row once more (from L2) with the threshold moved toward its k-th value
+      const float t2 = n < k ? pred * REFILTER_DOWN : pred * REFILTER_UP;
+      uint32_t km = 0;
+      for_each_score(p, row, len, [&](int j, float x) { fast_visit1(S, x, j, t2, km); });
+      km = __reduce_max_sync(0xffffffffu, km);
+      if (lane == 0) atomicMax(&S.kmax, km);
+      ConsumerSync::sync();
+      bool ov2;
+      if (list_size(S, ov2) >= k && !ov2) {
+        resolve_candidates<ConsumerSync>(p, S, __float_as_uint(t2) | 0x80000000u, thr, need_tie, &kth);
+        done = true;
+        refreshed = true;
+      }
+      ConsumerSync::sync();
+    }
+    if (!done) {
+      exact_select<ConsumerSync>(p, S, row, len, false, thr, need_tie);
+      kth = thr;
+      refreshed = true;
+    }
+    ConsumerSync::sync();
+    if (refreshed && tid == 0) M.pred_next = next_prediction(kth);  // a miss refreshes the prediction
+    write_row<ConsumerSync>(p, S, p.idx + r * p.idx_stride, (len + 31) >> 5, need_tie);
+    ConsumerSync::sync();
   }
-  if (p.pred_state && tid == 0) p.pred_state[blockIdx.x] = pred;
+  if (p.pred_state && tid == 0) p.pred_state[blockIdx.x] = M.pred_next;
 }
 
 }  // namespace topk

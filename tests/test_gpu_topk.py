@@ -44,6 +44,31 @@ def test_topk_random_rows(k, W):
     assert np.array_equal(gpu_topk(s, k), ora_topk(s, k))
 
 
+@pytest.mark.parametrize("W,k,rows", [(2048, 256, 9000), (26624, 512, 2400)])
+def test_topk_predictions_across_rows(W, k, rows):
+    """Enough rows that each selecting warp takes several in turn, so the
+    threshold predicted from one row meets the next: rows whose scale drops
+    (the prediction admits fewer than k), jumps (the candidate list
+    overflows), rows of heavy ties, rows whose boundary lies among zero
+    scores, constant rows and rows shorter than k.  The selection must not
+    depend on the prediction: it equals the oracle's exactly."""
+    rng = np.random.default_rng(W + k)
+    s = np.abs(rng.normal(size=(rows, W))).astype(np.float32) * 3
+    r = np.arange(rows)
+    s[r % 7 == 3] *= np.float32(0.3)
+    s[r % 11 == 5] *= np.float32(5.0)
+    tie_rows = r % 13 == 0
+    s[tie_rows] = np.round(s[tie_rows] * 2) / 2
+    few = r % 17 == 1
+    s[few] = np.where(rng.random(size=(int(few.sum()), W)) < 0.95, 0.0, s[few])
+    s[r % 19 == 2] = 2.5
+    s[rng.random(size=s.shape) < 0.01] = -np.inf
+    lengths = np.full(rows, W, dtype=np.int32)
+    short = r % 23 == 4
+    lengths[short] = rng.integers(0, k + 5, size=int(short.sum()))
+    assert np.array_equal(gpu_topk(s, k, lengths), ora_topk(s, k, lengths))
+
+
 def test_topk_ties_signed_zero_negative_and_nan():
     rng = np.random.default_rng(1)
     W, k = 3000, 300

@@ -24,6 +24,11 @@
 //  * Each lane streams its part of the keys with 16-byte non-caching global
 //    loads straight into registers (4 tiles = 256 bytes per lane in flight),
 //    in the operand layout of mma.sync.m16n8k16 (B = 16 features x 8 keys).
+//    Two loop forms (template PIPE): one batch of 4 tiles loaded, then
+//    multiplied; or two half-batches alternating, the next one's loads issued
+//    before the current one's math (the same bytes in flight, chosen at
+//    launch: the fp8 cache always, bf16 / fp16 when warps get at most one
+//    half-batch each).
 //  * The request's query rows (4 tokens x 4 heads = M 16) stay in registers
 //    as the A operand.  Features are visited in a permuted order, the same for
 //    queries and keys, so that every load instruction reads whole 32-byte
@@ -48,6 +53,8 @@
 #pragma once
 
 #include <cuda_fp16.h>
+
+#include <type_traits>
 
 #include "sm100.cuh"
 
@@ -230,7 +237,7 @@ __device__ __forceinline__ void page_of(const Params& p, int n, int& lp, int& ro
   }
 }
 
-template <Fmt F, bool GEN>
+template <Fmt F, bool GEN, bool PIPE>
 __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) {
   constexpr bool FP8 = F == Fmt::E4M3;
   constexpr int NB = FP8 ? 2 * BATCH : BATCH;  // tiles in flight per warp
@@ -437,94 +444,88 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
   };
   fetch_entries();
 
-  while (left > 0) {
-    const int cnt = (int)min((uint32_t)min(min(NB, nt_b - j), 32 - (j - j0)), left);
-    uint4 kv[FP8 ? 1 : NB][4];   // bf16: chunk i = 16 bytes
-    uint2 kv8[FP8 ? NB : 1][4];  // fp8: chunk i = 8 bytes
-    uint32_t valid = 0;  // bit u: the page of key g of tile u (this lane's loads) is valid
-#pragma unroll
-    for (int u = 0; u < NB; ++u) {
-      // keys past the request's pages (logical page >= max_pages) and
-      // entries outside the pool are invalid
-      int lp, row;
-      page_of<GEN>(p, (j + u) * TILE + g, lp, row);
-      const int src = GEN ? (lp - lp0) & 31 : (j - j0 + u) & 31;
-      const int ent = __shfl_sync(0xffffffffu, entry, src);
-      const bool ok = lp < p.max_pages && ent >= 0 && (int64_t)ent < p.num_pages;
-      valid |= ok ? 1u << u : 0u;
-      const int64_t off = (int64_t)ent * p.k_page_stride + (int64_t)row * p.k_row_stride;
-      if constexpr (FP8) {
-        if (u < cnt && ok) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) kv8[u][i] = ld_stream8(p.k8 + off + 8 * (c + 4 * i));
+  if constexpr (PIPE) {
+    // Two half-batches alternate: the loads of the next one go out before the
+    // math of the current one, so a warp always has keys in flight while it
+    // multiplies.  A batch never leaves its request; at a request boundary the
+    // pipeline drains, the next request's queries load, and it restarts.
+    constexpr int HB = NB / 2;  // tiles per half-batch
+    using KV = typename std::conditional<FP8, uint2, uint4>::type;
+    auto issue = [&](KV (&kv)[HB][4], int& jb, int& cnt, uint32_t& valid) {
+      cnt = (int)min((uint32_t)min(min(HB, nt_b - j), 32 - (j - j0)), left);
+      jb = j;
+      valid = 0;
+  #pragma unroll
+      for (int u = 0; u < HB; ++u) {
+        int lp, row;
+        page_of<GEN>(p, (j + u) * TILE + g, lp, row);
+        const int src = GEN ? (lp - lp0) & 31 : (j - j0 + u) & 31;
+        const int ent = __shfl_sync(0xffffffffu, entry, src);
+        const bool ok = lp < p.max_pages && ent >= 0 && (int64_t)ent < p.num_pages;
+        valid |= ok ? 1u << u : 0u;
+        const int64_t off = (int64_t)ent * p.k_page_stride + (int64_t)row * p.k_row_stride;
+        if constexpr (FP8) {
+          if (u < cnt && ok) {
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) kv[u][i] = ld_stream8(p.k8 + off + 8 * (c + 4 * i));
+          } else {
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) kv[u][i] = make_uint2(0, 0);
+          }
         } else {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) kv8[u][i] = make_uint2(0, 0);
-        }
-      } else {
-        if (u < cnt && ok) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) kv[u][i] = ld_stream16(p.k_cache + off + 8 * (c + 4 * i));
-        } else {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) kv[u][i] = make_uint4(0, 0, 0, 0);
+          if (u < cnt && ok) {
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) kv[u][i] = ld_stream16(p.k_cache + off + 8 * (c + 4 * i));
+          } else {
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) kv[u][i] = make_uint4(0, 0, 0, 0);
+          }
         }
       }
-    }
-    // validity of the key this lane stores (key 2c + lane / 16), held by the
-    // lanes that loaded it (4 * key .. 4 * key + 3); uniform over a tile
-    // when pages hold whole tiles
-    const uint32_t vst = GEN ? __shfl_sync(0xffffffffu, valid, key << 2) : valid;
-    const int vis = t < p.Q ? visible_of(L, p.Q, t) : 0;
-    const int jb = j;
-    j += cnt;
-    left -= (uint32_t)cnt;
-    // next request or next 32 tiles: issue those loads before the math
-    if (left > 0) {
-      if (j == nt_b) {
-        do {
-          ++b;
-        } while (pfx(b + 1) == pfx(b));
-        j = 0;
-        j0 = 0;
-        nt_b = (int)(pfx(b + 1) - pfx(b));
-        fetch_entries();
-      } else if (j - j0 == 32) {
-        j0 = j;
-        fetch_entries();
+      j += cnt;
+      left -= (uint32_t)cnt;
+      if (left > 0) {
+        if (j == nt_b) {
+          do {
+            ++b;
+          } while (pfx(b + 1) == pfx(b));
+          j = 0;
+          j0 = 0;
+          nt_b = (int)(pfx(b + 1) - pfx(b));
+          fetch_entries();
+        } else if (j - j0 == 32) {
+          j0 = j;
+          fetch_entries();
+        }
       }
-    }
-    // the MMA chains of four tiles interleaved by k-step: four independent
-    // accumulators keep the tensor pipe busy instead of waiting on one chain
-#pragma unroll
-    for (int u0 = 0; u0 < NB; u0 += BATCH) {
-      float d[BATCH][4];
-#pragma unroll
-      for (int v = 0; v < BATCH; ++v) d[v][0] = d[v][1] = d[v][2] = d[v][3] = 0.f;
-#pragma unroll
+    };
+    auto compute = [&](const KV (&kv)[HB][4], int jb, int cnt, uint32_t valid) {
+      const uint32_t vst = GEN ? __shfl_sync(0xffffffffu, valid, key << 2) : valid;
+      const int vis = t < p.Q ? visible_of(L, p.Q, t) : 0;
+      float d[HB][4];
+  #pragma unroll
+      for (int v = 0; v < HB; ++v) d[v][0] = d[v][1] = d[v][2] = d[v][3] = 0.f;
+  #pragma unroll
       for (int s = 0; s < 8; ++s) {
-#pragma unroll
-        for (int v = 0; v < BATCH; ++v) {
+  #pragma unroll
+        for (int v = 0; v < HB; ++v) {
           if constexpr (FP8) {
-            // words 2s, 2s + 1 = bytes 0-3 (s even) or 4-7 (s odd) of chunk s / 2
-            const uint32_t four = (s & 1) ? kv8[u0 + v][s >> 1].y : kv8[u0 + v][s >> 1].x;
+            const uint32_t four = (s & 1) ? kv[v][s >> 1].y : kv[v][s >> 1].x;
             uint32_t b0, b1;
             e4m3x4_to_f16x2x2(four, b0, b1);
             mma_f16_16816(d[v], qa[s], b0, b1);
           } else if constexpr (F == Fmt::F16) {
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[u0 + v]);
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[v]);
             mma_f16_16816(d[v], qa[s], w[2 * s], w[2 * s + 1]);
           } else {
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[u0 + v]);
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[v]);
             mma_bf16_16816(d[v], qa[s], w[2 * s], w[2 * s + 1]);
           }
         }
       }
-#pragma unroll
-      for (int v = 0; v < BATCH; ++v) {
-        const int u = u0 + v;
-        if (u < cnt) {
-          // d0/d1: head h, keys 2c and 2c+1; d2/d3: head h + 2
+  #pragma unroll
+      for (int v = 0; v < HB; ++v) {
+        if (v < cnt) {
           float s0, s1;
           if constexpr (FP8) {
             s0 = fmaxf(d[v][0], 0.f) * up0 + fmaxf(d[v][2], 0.f) * up1;
@@ -535,18 +536,147 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) 
           }
           s0 += __shfl_xor_sync(0xffffffffu, s0, 16);  // the other two heads
           s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-          const int n = (jb + u) * TILE + key;
+          const int n = (jb + v) * TILE + key;
           if (t < p.Q && n < p.W) {
             const float sc = p.scale * ((lane >> 4) ? s1 : s0);
-            p.out[(int64_t)ob * p.out_sb + (int64_t)t * p.out_st + n] = ((vst >> u) & 1u) && n < vis ? sc : -INFINITY;
+            p.out[(int64_t)ob * p.out_sb + (int64_t)t * p.out_st + n] = ((vst >> v) & 1u) && n < vis ? sc : -INFINITY;
           }
         }
       }
-    }
-    if (ob != b) {
+    };
+    KV kvA[HB][4], kvB[HB][4];
+    int jA = 0, cA = 0, jB = 0, cB = 0;
+    uint32_t vA = 0, vB = 0;
+    issue(kvA, jA, cA, vA);
+    while (true) {
+      bool more = left > 0 && b == ob;
+      if (more) issue(kvB, jB, cB, vB);
+      compute(kvA, jA, cA, vA);
+      if (more) {
+        more = left > 0 && b == ob;
+        if (more) issue(kvA, jA, cA, vA);
+        compute(kvB, jB, cB, vB);
+        if (more) continue;
+      }
+      if (left == 0) break;
+      // the next request: its queries, then a fresh pipeline
       ob = b;
       L = __ldg(p.seq_lens + b);
       load_queries<F>(p, b, lane, qa, up0, up1);
+      issue(kvA, jA, cA, vA);
+    }
+  } else {
+    while (left > 0) {
+      const int cnt = (int)min((uint32_t)min(min(NB, nt_b - j), 32 - (j - j0)), left);
+      uint4 kv[FP8 ? 1 : NB][4];   // bf16: chunk i = 16 bytes
+      uint2 kv8[FP8 ? NB : 1][4];  // fp8: chunk i = 8 bytes
+      uint32_t valid = 0;  // bit u: the page of key g of tile u (this lane's loads) is valid
+  #pragma unroll
+      for (int u = 0; u < NB; ++u) {
+        // keys past the request's pages (logical page >= max_pages) and
+        // entries outside the pool are invalid
+        int lp, row;
+        page_of<GEN>(p, (j + u) * TILE + g, lp, row);
+        const int src = GEN ? (lp - lp0) & 31 : (j - j0 + u) & 31;
+        const int ent = __shfl_sync(0xffffffffu, entry, src);
+        const bool ok = lp < p.max_pages && ent >= 0 && (int64_t)ent < p.num_pages;
+        valid |= ok ? 1u << u : 0u;
+        const int64_t off = (int64_t)ent * p.k_page_stride + (int64_t)row * p.k_row_stride;
+        if constexpr (FP8) {
+          if (u < cnt && ok) {
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) kv8[u][i] = ld_stream8(p.k8 + off + 8 * (c + 4 * i));
+          } else {
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) kv8[u][i] = make_uint2(0, 0);
+          }
+        } else {
+          if (u < cnt && ok) {
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) kv[u][i] = ld_stream16(p.k_cache + off + 8 * (c + 4 * i));
+          } else {
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) kv[u][i] = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+      // validity of the key this lane stores (key 2c + lane / 16), held by the
+      // lanes that loaded it (4 * key .. 4 * key + 3); uniform over a tile
+      // when pages hold whole tiles
+      const uint32_t vst = GEN ? __shfl_sync(0xffffffffu, valid, key << 2) : valid;
+      const int vis = t < p.Q ? visible_of(L, p.Q, t) : 0;
+      const int jb = j;
+      j += cnt;
+      left -= (uint32_t)cnt;
+      // next request or next 32 tiles: issue those loads before the math
+      if (left > 0) {
+        if (j == nt_b) {
+          do {
+            ++b;
+          } while (pfx(b + 1) == pfx(b));
+          j = 0;
+          j0 = 0;
+          nt_b = (int)(pfx(b + 1) - pfx(b));
+          fetch_entries();
+        } else if (j - j0 == 32) {
+          j0 = j;
+          fetch_entries();
+        }
+      }
+      // the MMA chains of four tiles interleaved by k-step: four independent
+      // accumulators keep the tensor pipe busy instead of waiting on one chain
+  #pragma unroll
+      for (int u0 = 0; u0 < NB; u0 += BATCH) {
+        float d[BATCH][4];
+  #pragma unroll
+        for (int v = 0; v < BATCH; ++v) d[v][0] = d[v][1] = d[v][2] = d[v][3] = 0.f;
+  #pragma unroll
+        for (int s = 0; s < 8; ++s) {
+  #pragma unroll
+          for (int v = 0; v < BATCH; ++v) {
+            if constexpr (FP8) {
+              // words 2s, 2s + 1 = bytes 0-3 (s even) or 4-7 (s odd) of chunk s / 2
+              const uint32_t four = (s & 1) ? kv8[u0 + v][s >> 1].y : kv8[u0 + v][s >> 1].x;
+              uint32_t b0, b1;
+              e4m3x4_to_f16x2x2(four, b0, b1);
+              mma_f16_16816(d[v], qa[s], b0, b1);
+            } else if constexpr (F == Fmt::F16) {
+              const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[u0 + v]);
+              mma_f16_16816(d[v], qa[s], w[2 * s], w[2 * s + 1]);
+            } else {
+              const uint32_t* w = reinterpret_cast<const uint32_t*>(kv[u0 + v]);
+              mma_bf16_16816(d[v], qa[s], w[2 * s], w[2 * s + 1]);
+            }
+          }
+        }
+  #pragma unroll
+        for (int v = 0; v < BATCH; ++v) {
+          const int u = u0 + v;
+          if (u < cnt) {
+            // d0/d1: head h, keys 2c and 2c+1; d2/d3: head h + 2
+            float s0, s1;
+            if constexpr (FP8) {
+              s0 = fmaxf(d[v][0], 0.f) * up0 + fmaxf(d[v][2], 0.f) * up1;
+              s1 = fmaxf(d[v][1], 0.f) * up0 + fmaxf(d[v][3], 0.f) * up1;
+            } else {
+              s0 = fmaxf(d[v][0], 0.f) + fmaxf(d[v][2], 0.f);
+              s1 = fmaxf(d[v][1], 0.f) + fmaxf(d[v][3], 0.f);
+            }
+            s0 += __shfl_xor_sync(0xffffffffu, s0, 16);  // the other two heads
+            s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+            const int n = (jb + u) * TILE + key;
+            if (t < p.Q && n < p.W) {
+              const float sc = p.scale * ((lane >> 4) ? s1 : s0);
+              p.out[(int64_t)ob * p.out_sb + (int64_t)t * p.out_st + n] = ((vst >> u) & 1u) && n < vis ? sc : -INFINITY;
+            }
+          }
+        }
+      }
+      if (ob != b) {
+        ob = b;
+        L = __ldg(p.seq_lens + b);
+        load_queries<F>(p, b, lane, qa, up0, up1);
+      }
     }
   }
 }

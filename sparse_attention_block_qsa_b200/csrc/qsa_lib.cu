@@ -130,12 +130,16 @@ qsa_status_t device_info(int* sms) {
       const void* fn;
       size_t bytes;
     } kernels[] = {
-        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::BF16, false>), qsa::decode::SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::BF16, true>), qsa::decode::SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::F16, false>), qsa::decode::SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::F16, true>), qsa::decode::SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::E4M3, false>), qsa::decode::SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::E4M3, true>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::BF16, false, false>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::BF16, true, false>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::BF16, false, true>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::BF16, true, true>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::F16, false, false>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::F16, true, false>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::F16, false, true>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::F16, true, true>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::E4M3, false, true>), qsa::decode::SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::decode::decode_kernel<qsa::decode::Fmt::E4M3, true, true>), qsa::decode::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel<false>), qsa::prefill::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::prefill::prefill_kernel<true>), qsa::prefill::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::attn::attn_kernel), qsa::attn::SMEM_BYTES},
@@ -434,13 +438,31 @@ qsa_status_t qsa_selftest_bounded_wait(uint64_t timeout_ns, int32_t arrive, void
 // Every format: E4M3 keys take 1 byte per element (strides multiples of 16)
 // and are scaled by k_scale; bf16 and fp16 keys take 2 (k_scale == 1).
 extern "C++" {
-template <qsa::decode::Fmt F, bool GEN>
+template <qsa::decode::Fmt F, bool GEN, bool PIPE>
 static void launch_decode(int sms, const qsa::decode::Params& p, cudaStream_t stream, bool pdl) {
   if (pdl)
-    launch_pdl(qsa::decode::decode_kernel<F, GEN>, dim3(sms), dim3(qsa::decode::NUM_THREADS), qsa::decode::SMEM_BYTES,
-               stream, p);
+    launch_pdl(qsa::decode::decode_kernel<F, GEN, PIPE>, dim3(sms), dim3(qsa::decode::NUM_THREADS),
+               qsa::decode::SMEM_BYTES, stream, p);
   else
-    qsa::decode::decode_kernel<F, GEN><<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES, stream>>>(p);
+    qsa::decode::decode_kernel<F, GEN, PIPE><<<sms, qsa::decode::NUM_THREADS, qsa::decode::SMEM_BYTES, stream>>>(p);
+}
+
+// The two-half-batch loop: always for the fp8 cache (its widening is the
+// longest step between batches); for bf16 / fp16 keys when no warp gets more
+// than one half-batch (measured on B200: fp8 16 x 4 long contexts 15.4 ->
+// 13.3 us, 16 x 1 8.2 -> 6.6 us; bf16 1 x 1 4.0 -> 3.5 us, but bf16 16 x 4
+// 13.2 -> 14.3 us).
+template <qsa::decode::Fmt F>
+static void launch_decode_fmt(int sms, const qsa::decode::Params& p, cudaStream_t stream, bool pdl, bool pow2,
+                              bool pipe) {
+  if constexpr (F == qsa::decode::Fmt::E4M3) {
+    pow2 ? launch_decode<F, false, true>(sms, p, stream, pdl) : launch_decode<F, true, true>(sms, p, stream, pdl);
+  } else {
+    if (pipe)
+      pow2 ? launch_decode<F, false, true>(sms, p, stream, pdl) : launch_decode<F, true, true>(sms, p, stream, pdl);
+    else
+      pow2 ? launch_decode<F, false, false>(sms, p, stream, pdl) : launch_decode<F, true, false>(sms, p, stream, pdl);
+  }
 }
 }
 
@@ -542,12 +564,14 @@ static qsa_status_t decode_common(const void* q, int64_t q_stride_b, int64_t q_s
     p.out = out + (int64_t)b0 * out_stride_b;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     using qsa::decode::Fmt;
+    const bool pipe = (int64_t)p.B * tiles_per_req <=
+                      (int64_t)sms * qsa::decode::WARPS * (qsa::decode::BATCH / 2);  // at most one half-batch a warp
     if (fmt == Fmt::E4M3)
-      pow2 ? launch_decode<Fmt::E4M3, false>(sms, p, s, pdl) : launch_decode<Fmt::E4M3, true>(sms, p, s, pdl);
+      launch_decode_fmt<Fmt::E4M3>(sms, p, s, pdl, pow2, pipe);
     else if (fmt == Fmt::F16)
-      pow2 ? launch_decode<Fmt::F16, false>(sms, p, s, pdl) : launch_decode<Fmt::F16, true>(sms, p, s, pdl);
+      launch_decode_fmt<Fmt::F16>(sms, p, s, pdl, pow2, pipe);
     else
-      pow2 ? launch_decode<Fmt::BF16, false>(sms, p, s, pdl) : launch_decode<Fmt::BF16, true>(sms, p, s, pdl);
+      launch_decode_fmt<Fmt::BF16>(sms, p, s, pdl, pow2, pipe);
     st = launch_status("decode kernel");
     if (st != QSA_OK) return st;
   }

@@ -244,6 +244,14 @@ def test_decode_fp8_many_requests():
     run_case_fp8(_many(1500, 4, 16, seed=99))
 
 
+def test_decode_many_short_requests():
+    """2000 requests of at most 60 tokens: every warp gets at most one
+    half-batch, so the bf16 launch takes the two-half-batch loop, and warps
+    cross from one request to the next (more than half as many requests as
+    warps)."""
+    run_case(_many(2000, 2, 8, seed=2002, max_len=60))
+
+
 # ---------------------------------------------------------------- large pages, dense and padded rows
 
 @pytest.mark.parametrize("ps", [32, 64, 128, 1024])

@@ -824,6 +824,8 @@ def measure(cfg: int, args, world: int, rank: int, local: int, cpu_budget_s: flo
         fused = b.time_fused()
         if fused is not None:
             extra["fused_l2_workspace"] = fused
+            # the same call with a workspace of 512 MiB: fewer, fuller chunks
+            extra["fused_512mib_workspace"] = b.time_fused(workspace_mib=512)
     e2e_s = max_over_ranks(time_e2e(b, args.steps, 3, world), world)
     from sparse_attention_block_qsa_b200 import device_error
     dev_err = device_error()
@@ -946,7 +948,7 @@ def main():
                 "roofline": head["roofline"], "e2e": head["e2e"],
                 "gpu_launches": sum(r["gpu_launches"] for r in records.values()),
                 "clocks": head["clocks"], "device_error": max(r["device_error"] for r in records.values())}
-        for key in ("kernels", "fused_l2_workspace", "all_inputs_cold_us", "cpu_baseline"):
+        for key in ("kernels", "fused_l2_workspace", "fused_512mib_workspace", "all_inputs_cold_us", "cpu_baseline"):
             if key in head:
                 line[key] = head[key]
         if len(configs) > 1:

@@ -247,8 +247,12 @@ qsa_status_t qsa_topk(const float* scores, int64_t score_stride, const int32_t* 
  * and hold 4096 bytes of selection state plus at least min(T, 64) rows of W
  * floats; qsa_prefill_topk_workspace_size gives the size that needs a single
  * chunk.
- * A workspace of a few tens of MB lets the chunk's scores stay in the
- * B200's 126 MB L2 between the two kernels.
+ * A workspace of a few tens of MB keeps each chunk's scores in the B200's
+ * 126 MB L2 between the two kernels, but leaves each chunk a few hundred
+ * rows for 148 SMs.  Measured on B200 for 4 x 4,096 rows of 26,624 keys,
+ * top-512: a 64 MiB workspace 1.96 ms per call, 512 MiB 1.26 ms, and the two
+ * separate calls over every row 1.13 ms.  The workspace bounds memory; larger
+ * chunks are faster.
  */
 qsa_status_t qsa_mqa_prefill_topk(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,
                                   int64_t k_stride, int64_t Nk, const int32_t* ks, const int32_t* ke, int64_t T,

@@ -43,8 +43,9 @@
 //
 // fp8 E4M3 cache (vLLM qsa_cache.py, the state backend's fp8 cache dtypes;
 // vLLM qsa_prepare.py, "_to_dst_dtype": stored = e4m3(bf16(k) / k_scale)):
-// a lane reads 8 bytes per chunk instead of 16, with twice the tiles in
-// flight (the same 256 bytes per lane).  Every E4M3 value is exact in fp16,
+// a lane reads 8 bytes per chunk instead of 16, with 6 tiles in flight as
+// two halves of 3 (192 bytes per lane; 8 tiles spill registers and measured
+// slower, 4 keep too few bytes in flight).  Every E4M3 value is exact in fp16,
 // so keys are widened with one conversion per pair and the MMA runs on fp16.
 // The query rows are made fp16 exactly: each row is multiplied by the power
 // of two that puts its largest magnitude in [2^15, 2^16) (exact for every
@@ -62,7 +63,7 @@ namespace qsa {
 namespace decode {
 
 constexpr int TILE = 8;                 // keys per tile (mma.sync N)
-constexpr int BATCH = 4;                // tiles in flight per warp (bf16 keys; fp8 keys: 2 * BATCH)
+constexpr int BATCH = 4;                // tiles in flight per warp (bf16 and fp16 keys)
 constexpr int WARPS = 16;
 constexpr int NUM_THREADS = WARPS * 32;
 constexpr int MAX_B = 8192;             // requests per launch (prefix in shared memory)
@@ -240,7 +241,7 @@ __device__ __forceinline__ void page_of(const Params& p, int n, int& lp, int& ro
 template <Fmt F, bool GEN, bool PIPE>
 __global__ void __launch_bounds__(NUM_THREADS, 1) decode_kernel(const Params p) {
   constexpr bool FP8 = F == Fmt::E4M3;
-  constexpr int NB = FP8 ? 2 * BATCH : BATCH;  // tiles in flight per warp
+  constexpr int NB = FP8 ? 6 : BATCH;  // tiles in flight per warp (fp8: two halves of 3)
   extern __shared__ int32_t prefix[];  // prefix[b]: tiles before request b
   __shared__ uint32_t red[WARPS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

@@ -450,7 +450,7 @@ static void launch_decode(int sms, const qsa::decode::Params& p, cudaStream_t st
 // The two-half-batch loop: always for the fp8 cache (its widening is the
 // longest step between batches); for bf16 / fp16 keys when no warp gets more
 // than one half-batch (measured on B200: fp8 16 x 4 long contexts 15.4 ->
-// 13.3 us, 16 x 1 8.2 -> 6.6 us; bf16 1 x 1 4.0 -> 3.5 us, but bf16 16 x 4
+// 12.8 us, 16 x 1 8.2 -> 6.3 us; bf16 1 x 1 4.0 -> 3.5 us, but bf16 16 x 4
 // 13.2 -> 14.3 us).
 template <qsa::decode::Fmt F>
 static void launch_decode_fmt(int sms, const qsa::decode::Params& p, cudaStream_t stream, bool pdl, bool pow2,

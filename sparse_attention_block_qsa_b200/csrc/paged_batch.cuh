@@ -14,7 +14,8 @@
 //    with TMA tiles.  Keys are small next to the scores they feed (256 bytes
 //    per key against 4 bytes per row), so the copy costs little.
 //  * fixup_kernel: the scores of keys whose page is missing become -inf
-//    (one CTA per prefill request; nothing to do when every page is there).
+//    (one CTA per prefill request, one page entry per lane; nothing to do
+//    when every page is there).
 #pragma once
 
 #include "sm100.cuh"
@@ -141,7 +142,10 @@ __global__ void __launch_bounds__(THREADS) gather_kernel(const Params p) {
   }
 }
 
-// One CTA per prefill request: -inf over the scores of keys whose page is missing.
+// One CTA per prefill request: -inf over the scores of keys whose page is
+// missing.  Each lane checks one page entry, so a warp covers 32 pages per
+// round trip; the (rare) missing pages are then handled one at a time by the
+// whole warp.
 __global__ void __launch_bounds__(THREADS) fixup_kernel(const Params p) {
   pdl_wait_then_release();
   const int r = p.D + blockIdx.x;
@@ -151,15 +155,23 @@ __global__ void __launch_bounds__(THREADS) fixup_kernel(const Params p) {
   const int first = __ldg(p.cu + r);
   const int qlen = __ldg(p.cu + r + 1) - first;
   const int pages = (n_r + p.page_size - 1) / p.page_size;
-  for (int lp = warp; lp < pages; lp += THREADS / 32) {
-    const int page = lp < p.max_pages ? __ldg(p.page_table + (int64_t)r * p.pt_stride + lp) : -1;
-    if (page >= 0 && (int64_t)page < p.num_pages) continue;
-    const int k0 = lp * p.page_size, k1 = min(k0 + p.page_size, n_r);
-    for (int i = 0; i < qlen; ++i) {
-      const int pos = L - qlen + i;
-      const int vis = max(0, min((pos + 1) >> 2, L >> 2));
-      float* row = p.out + (int64_t)(first + i) * p.out_stride;
-      for (int j = k0 + lane; j < min(k1, vis); j += 32) row[j] = -INFINITY;
+  for (int lp0 = warp * 32; lp0 < pages; lp0 += THREADS) {
+    const int lp = lp0 + lane;
+    bool missing = false;
+    if (lp < pages) {
+      const int page = lp < p.max_pages ? __ldg(p.page_table + (int64_t)r * p.pt_stride + lp) : -1;
+      missing = !(page >= 0 && (int64_t)page < p.num_pages);
+    }
+    unsigned m = __ballot_sync(0xffffffffu, missing);
+    while (m) {
+      const int k0 = (lp0 + __ffs(m) - 1) * p.page_size, k1 = min(k0 + p.page_size, n_r);
+      m &= m - 1;
+      for (int i = 0; i < qlen; ++i) {
+        const int pos = L - qlen + i;
+        const int vis = max(0, min((pos + 1) >> 2, L >> 2));
+        float* row = p.out + (int64_t)(first + i) * p.out_stride;
+        for (int j = k0 + lane; j < min(k1, vis); j += 32) row[j] = -INFINITY;
+      }
     }
   }
 }

@@ -58,6 +58,8 @@ def test_mixed_batch_missing_pages_and_narrow_width():
     pt[2, 1] = -1                                  # prefill request pages: missing and out of the pool
     pt[3, 10] = b.k_cache.shape[0] + 2
     pt[3, 0] = -1
+    pt[3, 40] = -1                                 # pages past the first 32 (another lane group)
+    pt[3, 93] = -1                                 # the last, partly used page of the 1,500 keys
     run_and_check(b, page_table=pt)
 
 

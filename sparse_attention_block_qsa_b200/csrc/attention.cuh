@@ -9,10 +9,11 @@
 //  * attn_kernel: split-KV sparse attention.  One CTA per (row, KV head,
 //    split of the row's token list).  The row's query heads of one KV head
 //    (up to 16; 12 for the canonical 24 / 2 geometry) are the M = 16 side of
-//    mma.sync.m16n8k16 and stay in registers.  Each 32-entry chunk of the
-//    token list is gathered row by row (512-byte K and V rows found through
-//    the page table) with 16-byte cp.async copies into a 3-stage shared-memory
-//    ring (XOR-swizzled 16-byte units, so ldmatrix reads are conflict-free;
+//    mma.sync.m16n8k16, read from shared memory for every chunk (so three
+//    CTAs fit an SM).  Each 32-entry chunk of the token list is gathered row
+//    by row (512-byte K and V rows found through the page table) with
+//    16-byte cp.async copies into a 2-stage shared-memory ring per CTA
+//    (XOR-swizzled 16-byte units, so ldmatrix reads are conflict-free;
 //    masked entries are zero-filled).  Warp w scores the chunk's tokens
 //    8w .. 8w + 7 against all heads, the chunk maximum is exchanged through
 //    shared memory, and the probabilities (bf16) are written to shared memory
@@ -37,7 +38,7 @@ namespace attn {
 
 constexpr int D = 256;            // head dimension
 constexpr int CHUNK = 32;         // token-list entries per pipeline stage
-constexpr int STAGES = 3;
+constexpr int STAGES = 2;
 constexpr int WARPS = 4;
 constexpr int THREADS = WARPS * 32;
 constexpr int MAX_GROUP = 16;     // query heads per KV head (the MMA's M)
@@ -201,7 +202,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-__global__ void __launch_bounds__(THREADS, 2) attn_kernel(const Params p) {
+__global__ void __launch_bounds__(THREADS, 3) attn_kernel(const Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* q_s = smem;
   uint8_t* kv_s = smem + Q_BYTES;                                   // stage s: K at 2s, V at 2s + 1
@@ -298,17 +299,13 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(const Params p) {
     cp_async_commit();
   }
 
-  // query fragments (A, 16 x 256): 16 k-steps of 16 features
-  uint32_t qa[16][4];
-  __syncthreads();
-  {
-    const uint32_t qb = smem_addr(q_s);
-    // ldmatrix x4: matrices (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15)
-    const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
-    const int khalf = lane >> 4;
-#pragma unroll
-    for (int s = 0; s < 16; ++s) ldsm_x4(qb + swz(row, 2 * s + khalf), qa[s][0], qa[s][1], qa[s][2], qa[s][3]);
-  }
+  // query fragments (A, 16 x 256) are read from shared memory for every
+  // chunk rather than held in registers (64 fewer registers: three CTAs per
+  // SM).  ldmatrix x4: matrices (rows 0-7, k 0-7), (rows 8-15, k 0-7),
+  // (rows 0-7, k 8-15), (rows 8-15, k 8-15).
+  const uint32_t qb = smem_addr(q_s);
+  const int q_row = (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int q_khalf = lane >> 4;
 
   const int g8 = lane >> 2, c4 = lane & 3;
   float m_run[2] = {-INFINITY, -INFINITY};  // rows g8, g8 + 8 (log2 units)
@@ -337,10 +334,12 @@ __global__ void __launch_bounds__(THREADS, 2) attn_kernel(const Params p) {
       const int q4 = lane >> 3;
 #pragma unroll
       for (int s2 = 0; s2 < 8; ++s2) {
-        uint32_t b0, b1, b2, b3;
+        uint32_t b0, b1, b2, b3, a0, a1, a2, a3, a4, a5, a6, a7;
         ldsm_x4(kb + swz(n, 4 * s2 + q4), b0, b1, b2, b3);
-        mma_bf16(sc, qa[2 * s2][0], qa[2 * s2][1], qa[2 * s2][2], qa[2 * s2][3], b0, b1);
-        mma_bf16(sc, qa[2 * s2 + 1][0], qa[2 * s2 + 1][1], qa[2 * s2 + 1][2], qa[2 * s2 + 1][3], b2, b3);
+        ldsm_x4(qb + swz(q_row, 4 * s2 + q_khalf), a0, a1, a2, a3);
+        ldsm_x4(qb + swz(q_row, 4 * s2 + 2 + q_khalf), a4, a5, a6, a7);
+        mma_bf16(sc, a0, a1, a2, a3, b0, b1);
+        mma_bf16(sc, a4, a5, a6, a7, b2, b3);
       }
     }
     // sc[0], sc[1]: row g8, tokens 8w + 2c4 + {0,1}; sc[2], sc[3]: row g8 + 8

@@ -384,13 +384,13 @@ std::mutex g_noalloc_mu;
 
 // Split-KV plan of the sparse attention: a row's token list is cut into
 // `splits` runs of `cps` 32-entry chunks, so that rows x KV heads x splits
-// gives the grid at most about 8 CTAs per SM of a 148-SM part (four waves of
-// two resident CTAs; rounded down so that the last wave is full; device
+// gives the grid at most about 9 CTAs per SM of a 148-SM part (three waves
+// of three resident CTAs; rounded down so that the last wave is full; device
 // independent, so the workspace size depends on the shapes only).
 void attn_splits(int64_t T, int32_t Hkv, int32_t width, int32_t* splits, int32_t* cps) {
   const int64_t chunks = std::max<int64_t>(1, ((int64_t)width + qsa::attn::CHUNK - 1) / qsa::attn::CHUNK);
   const int64_t pairs = std::max<int64_t>(1, T * Hkv);
-  int64_t sp = std::min<int64_t>(chunks, std::max<int64_t>(1, 1184 / pairs));
+  int64_t sp = std::min<int64_t>(chunks, std::max<int64_t>(1, 1332 / pairs));
   const int64_t per = (chunks + sp - 1) / sp;
   sp = (chunks + per - 1) / per;
   *splits = (int32_t)sp;

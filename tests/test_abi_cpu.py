@@ -240,9 +240,9 @@ def test_attention_rejects(kw, code):
 
 def test_attention_workspace_size():
     n = qsa.sparse_attention_workspace_size(64, 24, 2, 2051)
-    # 64 rows x 2 KV heads = 128 pairs -> floor(1184 / 128) = 9 splits of ceil(65 / 9) = 8
-    # of the 65 chunks of 32 entries; 12 heads x (256 + 2) floats per split
-    assert n == 64 * 2 * 9 * 12 * 258 * 4
+    # 64 rows x 2 KV heads = 128 pairs -> floor(1332 / 128) = 10 splits of ceil(65 / 10) = 7
+    # of the 65 chunks of 32 entries (ceil(65 / 7) = 10 runs); 12 heads x (256 + 2) floats per split
+    assert n == 64 * 2 * 10 * 12 * 258 * 4
     assert qsa.sparse_attention_workspace_size(0, 24, 2, 2051) == 0
     assert qsa.sparse_attention_workspace_size(4, 24, 5, 2051) == 0
 

@@ -178,17 +178,20 @@ class DecodeBench:
     kernel = "decode_kernel"
     bound = "hbm"
 
-    def __init__(self, cfg: int, dev: torch.device, seed: int, fp8: bool = False):
+    def __init__(self, cfg: int, dev: torch.device, seed: int, fp8: bool = False, page_size: int | None = None,
+                 f16: bool = False):
         import sparse_attention_block_qsa_b200 as qsa
         self.qsa = qsa
-        self.inp = wl.make_config(cfg, seed=seed)
+        self.inp = wl.make_config(cfg, seed=seed, page_size=page_size)
         d = self.inp
         self.fp8 = fp8
         self.k_scale = 1.0
         if fp8:   # the same keys in the fp8 E4M3 cache format
             d.k_cache, self.k_scale = wl.e4m3_cache(d.k_cache)
+        if f16:   # the same values as fp16 queries and keys
+            d.q, d.k_cache = d.q.to(torch.float16), d.k_cache.to(torch.float16)
         kb = d.k_cache.element_size()
-        self.name = d.name + ("_fp8" if fp8 else "")
+        self.name = d.name + ("_fp8" if fp8 else "") + ("_f16" if f16 else "")
         self.units = decode_bytes(d.seq_lens.tolist(), d.Q, 128 * kb)   # algorithmic bytes per step
         per_copy = d.q.numel() * 2 + d.k_cache.numel() * kb + d.B * d.Q * d.W * 4
         self.copies = max(2, math.ceil(2 * L2_BYTES / per_copy))
@@ -206,8 +209,9 @@ class DecodeBench:
         self.launches_per_step = 1
         self.h2d = d.q.numel() * 2 + d.k_cache.numel() * kb + (d.page_table.numel() + d.seq_lens.numel()) * 4
         self.d2h = d.B * d.Q * d.W * 4
-        self.dtype = "fp8e4m3 keys, bf16 queries" if fp8 else "bf16"
-        self.config = {"workload": self.name, "kv_cache_dtype": "fp8_e4m3" if fp8 else "bf16", "requests": d.B, "query_tokens": d.Q, "page_size": d.page_size,
+        self.dtype = "fp8e4m3 keys, bf16 queries" if fp8 else ("f16" if f16 else "bf16")
+        self.config = {"workload": self.name, "kv_cache_dtype": "fp8_e4m3" if fp8 else ("fp16" if f16 else "bf16"),
+                       "requests": d.B, "query_tokens": d.Q, "page_size": d.page_size,
                        "context_tokens": d.meta["context_tokens"], "W": d.W, "input_copies": self.copies,
                        "l2": f"steps rotate over {self.copies} copies of the key pool and output "
                              f"({self.copies * per_copy / 2**20:.0f} MiB > 2x L2); queries, lengths and page "
@@ -264,12 +268,16 @@ class PrefillBench:
     bound = "tensor"
     unit = "TFLOP/s"
 
-    def __init__(self, cfg: int, dev: torch.device, seed: int):
+    def __init__(self, cfg: int, dev: torch.device, seed: int, f16: bool = False):
         import sparse_attention_block_qsa_b200 as qsa
         self.qsa = qsa
         self.cfg = cfg
         self.inp = p = wl.make_config(cfg, seed=seed)
-        self.name = p.name
+        if f16:   # the same values as fp16 queries and keys
+            p.q, p.k = p.q.to(torch.float16), p.k.to(torch.float16)
+        self.f16 = f16
+        self.dtype = "f16" if f16 else "bf16"
+        self.name = p.name + ("_f16" if f16 else "")
         self.dev = dev
         self.q, self.k = p.q.to(dev), p.k.to(dev)
         self.cu, self.sl, self.ko = p.cu_seqlens_q.to(dev), p.seq_lens.to(dev), p.key_offsets.to(dev)
@@ -583,16 +591,20 @@ class MixedBench:
         oracle.decode(rows, b.k_cache, b.page_table[r:r + 1], cut, b.W, threads=threads)
 
 
-def make_bench(cfg: int, dev, seed: int, fp8: bool = False):
+def make_bench(cfg: int, dev, seed: int, fp8: bool = False, page_size: int | None = None, f16: bool = False):
     if fp8 and cfg not in (1, 2, 3):
         raise ValueError("the fp8 key cache applies to the decode configurations 1-3")
+    if page_size is not None and cfg not in (1, 2, 3):
+        raise ValueError("--page-size applies to the decode configurations 1-3")
+    if f16 and cfg not in (1, 2, 3, 4):
+        raise ValueError("--f16 applies to the decode configurations 1-3 and the prefill configuration 4")
     if cfg in (1, 2, 3):
-        return DecodeBench(cfg, dev, seed, fp8)
+        return DecodeBench(cfg, dev, seed, fp8, page_size, f16)
     if cfg == 6:
         return AttentionBench(cfg, dev, seed)
     if cfg == 7:
         return MixedBench(cfg, dev, seed)
-    return PrefillBench(cfg, dev, seed)
+    return PrefillBench(cfg, dev, seed, f16)
 
 
 # ------------------------------------------------------------------ timing
@@ -711,7 +723,7 @@ def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
     import oracle
-    inp_bench = _HostOnly(args.config or HEADLINE, args.kv_fp8)
+    inp_bench = _HostOnly(args.config or HEADLINE, args.kv_fp8, args.page_size, args.f16)
     threads = oracle.default_threads()
     frac, what = inp_bench.oracle_sample()
     for _ in range(args.warmup):
@@ -735,10 +747,11 @@ def run_reference(args, rank: int, world: int):
 class _HostOnly:
     """Inputs and accounting of a workload without any GPU state."""
 
-    def __init__(self, cfg: int, fp8: bool = False):
+    def __init__(self, cfg: int, fp8: bool = False, page_size: int | None = None, f16: bool = False):
         self.cfg = cfg
-        self.inp = wl.make_config(cfg)
+        self.inp = wl.make_config(cfg, page_size=page_size if cfg in (1, 2, 3) else None)
         self.fp8 = fp8 and cfg in (1, 2, 3)
+        self.f16 = f16 and cfg in (1, 2, 3, 4)
         self.k_scale = 1.0
         if cfg == 7:
             self.unit = "us"
@@ -752,18 +765,23 @@ class _HostOnly:
             d = self.inp
             if self.fp8:
                 d.k_cache, self.k_scale = wl.e4m3_cache(d.k_cache)
+            if self.f16:
+                d.q, d.k_cache = d.q.to(torch.float16), d.k_cache.to(torch.float16)
             self.units = decode_bytes(d.seq_lens.tolist(), d.Q, 128 * d.k_cache.element_size())
             self.unit = "GB/s"
-            self.config = {"workload": d.name + ("_fp8" if self.fp8 else ""),
-                           "kv_cache_dtype": "fp8_e4m3" if self.fp8 else "bf16", "requests": d.B,
-                           "query_tokens": d.Q, "page_size": d.page_size, "W": d.W}
+            self.config = {"workload": d.name + ("_fp8" if self.fp8 else "") + ("_f16" if self.f16 else ""),
+                           "kv_cache_dtype": "fp8_e4m3" if self.fp8 else ("fp16" if self.f16 else "bf16"),
+                           "requests": d.B, "query_tokens": d.Q, "page_size": d.page_size, "W": d.W}
         else:
             import oracle
             p = self.inp
+            if self.f16:
+                p.q, p.k = p.q.to(torch.float16), p.k.to(torch.float16)
             ks, ke = oracle.prefill_intervals(p.cu_seqlens_q, p.seq_lens, p.key_offsets)
             self.units = prefill_flops(ks, ke)
             self.unit = "TFLOP/s"
-            self.config = {"workload": p.name, "keys": p.Nk, "W": p.W}
+            self.topk = cfg == 5
+            self.config = {"workload": p.name + ("_f16" if self.f16 else ""), "keys": p.Nk, "W": p.W}
 
     def throughput(self, s):
         if self.unit == "us":
@@ -796,7 +814,9 @@ def measure(cfg: int, args, world: int, rank: int, local: int, cpu_budget_s: flo
     through the public binding; the oracle on the host cores (rank 0, N = 1).
     Returns rank 0's record (None on the other ranks)."""
     dev = torch.device("cuda", local)
-    b = make_bench(cfg, dev, seed=rank, fp8=args.kv_fp8 and cfg in (1, 2, 3))
+    b = make_bench(cfg, dev, seed=rank, fp8=args.kv_fp8 and cfg in (1, 2, 3),
+                   page_size=args.page_size if cfg in (1, 2, 3) else None,
+                   f16=args.f16 and cfg in (1, 2, 3, 4))
     for i in range(args.warmup):
         b.step(i)
     torch.cuda.synchronize()
@@ -853,7 +873,7 @@ def measure(cfg: int, args, world: int, rank: int, local: int, cpu_budget_s: flo
                         if peaks["source"] == "measured" else "fallback"}
             if b.bound == "tensor":
                 roofline["frac_of_burst"] = achieved / peaks["bf16_tflops"]
-        pub = None if args.kv_fp8 else PUBLISHED.get(cfg)
+        pub = None if (args.kv_fp8 or args.page_size or args.f16) else PUBLISHED.get(cfg)
         conf = dict(b.config)
         if pub:
             conf["published_reference"] = pub[2]
@@ -914,6 +934,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kv-fp8", action="store_true", help="decode over the fp8 E4M3 key cache")
+    ap.add_argument("--page-size", type=int, default=None,
+                    help="decode workloads over a pool of this page size (e.g. 196) instead of their own")
+    ap.add_argument("--f16", action="store_true", help="fp16 queries and keys (decode workloads and workload 4)")
     ap.add_argument("--soak", type=float, default=1.5, help="seconds of load before each timed region")
     args = ap.parse_args()
     if args.warmup < 3:

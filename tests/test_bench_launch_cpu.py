@@ -68,3 +68,20 @@ def test_two_replica_ranks_through_torchrun(tmp_path):
     assert res["world"] == 2 and res["slowest"] == pytest.approx(2e-3)
     one = bench.decode_bytes(__import__("workloads").make_config(2, seed=0).seq_lens.tolist(), 1)
     assert res["value"] == pytest.approx(one * 2 / 2e-3 / 1e9)
+
+
+@pytest.mark.parametrize("args", [["--config", "4"], ["--config", "5"], ["--config", "2", "--page-size", "196"],
+                                  ["--config", "4", "--f16"]])
+def test_reference_arm_runs_on_the_host(args):
+    """`bench.py --impl reference` times the oracle on the host cores (no GPU)
+    and prints one JSON line with the workload's name, unit and a positive
+    value, for the prefill workloads and the page-size / fp16 variants too."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3", *args], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    if "--page-size" in args:
+        assert line["config"]["workload"].endswith("_ps196")
+    if "--f16" in args:
+        assert line["config"]["workload"].endswith("_f16")

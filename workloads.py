@@ -235,16 +235,23 @@ def attention_block_sets(a: "AttentionInputs", n: int, seed: int) -> list:
     return out
 
 
-def make_config(idx: int, seed: int = 0):
+def make_config(idx: int, seed: int = 0, page_size: int | None = None):
+    """Workload idx; for the decode workloads 1-3, page_size (if given)
+    replaces the workload's page size (the same contexts, a pool of that
+    page size)."""
     name = CONFIG_NAMES[idx]
+    if page_size is not None:
+        if idx not in (1, 2, 3):
+            raise ValueError("a page size applies to the decode workloads 1-3")
+        name = name.rsplit("_ps", 1)[0] + f"_ps{page_size}"
     if idx == 1:
-        return make_decode(name, [2048], Q=1, page_size=16, seed=seed)
+        return make_decode(name, [2048], Q=1, page_size=page_size or 16, seed=seed)
     if idx == 2:
         ctx = lognormal_contexts(16, 1536, 43876, 16 * 10240, seed)
-        return make_decode(name, ctx, Q=1, page_size=64, seed=seed)
+        return make_decode(name, ctx, Q=1, page_size=page_size or 64, seed=seed)
     if idx == 3:
         ctx = lognormal_contexts(16, 3508, 102400, 16 * 51200, seed)
-        return make_decode(name, ctx, Q=4, page_size=64, seed=seed)
+        return make_decode(name, ctx, Q=4, page_size=page_size or 64, seed=seed)
     if idx == 4:
         return make_prefill(name, [8192], [50144], seed=seed)
     if idx == 5:

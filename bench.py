@@ -293,7 +293,7 @@ class PrefillBench:
         out_bytes = p.T * p.W * 4
         self.h2d = (p.q.numel() + p.k.numel()) * 2 + (p.cu_seqlens_q.numel() + 2 * p.seq_lens.numel()) * 4
         self.d2h = p.T * wl.TOPK_K * 4 if self.topk else out_bytes
-        self.config = {"workload": p.name, "sequences": len(p.meta["new_tokens"]),
+        self.config = {"workload": self.name, "sequences": len(p.meta["new_tokens"]),
                        "new_tokens": p.meta["new_tokens"], "prefix_tokens": p.meta["prefix_tokens"],
                        "keys": p.Nk, "W": p.W, "flop_per_step": self.units,
                        "l2": f"each step writes {out_bytes / 2**20:.0f} MiB of scores (> L2)"}
@@ -959,6 +959,13 @@ def main():
     records = {}
     for i, cfg in enumerate(configs):
         records[cfg] = measure(cfg, args, world, rank, local, cpu_budget_s=10.0 if i == 0 else 5.0)
+    # the default run also times the spec-decode workload over 196-row pages,
+    # the page size the vLLM PR's microbenchmarks use
+    variants = []
+    if not args.config and not (args.page_size or args.f16 or args.kv_fp8):
+        v = argparse.Namespace(**vars(args))
+        v.page_size = 196
+        variants.append(measure(HEADLINE, v, world, rank, local, cpu_budget_s=5.0))
 
     if rank == 0:
         head = records[configs[0]]
@@ -969,13 +976,14 @@ def main():
                 "config": head["config"],
                 "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                 "roofline": head["roofline"], "e2e": head["e2e"],
-                "gpu_launches": sum(r["gpu_launches"] for r in records.values()),
-                "clocks": head["clocks"], "device_error": max(r["device_error"] for r in records.values())}
+                "gpu_launches": sum(r["gpu_launches"] for r in list(records.values()) + variants),
+                "clocks": head["clocks"], "device_error": max(r["device_error"] for r in list(records.values()) + variants)}
         for key in ("kernels", "fused_l2_workspace", "fused_512mib_workspace", "all_inputs_cold_us", "cpu_baseline"):
             if key in head:
                 line[key] = head[key]
         if len(configs) > 1:
             line["configs"] = {records[c]["workload"]: records[c] for c in configs[1:]}
+            line["configs"].update({r["workload"]: r for r in variants})
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

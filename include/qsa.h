@@ -236,6 +236,32 @@ qsa_status_t qsa_topk(const float* scores, int64_t score_stride, const int32_t* 
                       int32_t W, int32_t k, int32_t* idx, int64_t idx_stride, void* stream);
 
 /*
+ * qsa_topk_ws - qsa_topk with a caller workspace: the same selection and
+ * result, computed in passes that stage each row's candidates in the
+ * workspace (a filter pass over the scores, a per-row selection on the
+ * staged candidates, an exact pass over the rows the first two cannot
+ * resolve), which is faster for many rows.
+ *
+ *   workspace        device memory of at least
+ *                    qsa_topk_workspace_size(rows, W, k) bytes, 256-byte
+ *                    aligned, not overlapping scores, lengths or idx.  Its
+ *                    contents on entry do not change the result; a workspace
+ *                    reused from one call to the next carries the selection's
+ *                    threshold predictions along, which only speeds the next
+ *                    call up.  Contents on return are undefined.
+ *   workspace_bytes  its size.
+ * Other arguments as for qsa_topk.  QSA_ERR_WORKSPACE when workspace_bytes
+ * is too small; rows whose start is not 16-byte aligned, or W not a multiple
+ * of 4, run as in qsa_topk (the workspace is then unused).
+ */
+qsa_status_t qsa_topk_ws(const float* scores, int64_t score_stride, const int32_t* lengths, int64_t rows,
+                         int32_t W, int32_t k, int32_t* idx, int64_t idx_stride, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace qsa_topk_ws needs (about 25.7 KB per row); 0 for rows <= 0. */
+size_t qsa_topk_workspace_size(int64_t rows, int32_t W, int32_t k);
+
+/*
  * qsa_mqa_prefill_topk - prefill scores followed by per-row top-k, without
  * materialising more than one workspace of scores at a time.
  *

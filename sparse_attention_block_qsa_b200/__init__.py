@@ -11,9 +11,9 @@ that library.
 from ._abi import (SCALE, QSAError, device_error, expand_block_indices, lib, mqa_decode, mqa_decode_fp8,
                    mqa_paged_batch, mqa_prefill, mqa_prefill_topk, mqa_prefill_topk_noalloc,
                    paged_batch_workspace_size, prefill_intervals, prefill_topk_workspace_size, selftest_bounded_wait, sparse_attention,
-                   sparse_attention_workspace_size, topk)
+                   sparse_attention_workspace_size, topk, topk_workspace_size)
 
 __all__ = ["SCALE", "QSAError", "device_error", "expand_block_indices", "lib", "mqa_decode", "mqa_decode_fp8",
            "mqa_paged_batch", "mqa_prefill", "mqa_prefill_topk", "paged_batch_workspace_size", "mqa_prefill_topk_noalloc", "prefill_intervals",
            "prefill_topk_workspace_size", "selftest_bounded_wait", "sparse_attention",
-           "sparse_attention_workspace_size", "topk"]
+           "sparse_attention_workspace_size", "topk", "topk_workspace_size"]

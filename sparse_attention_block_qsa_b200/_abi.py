@@ -36,6 +36,8 @@ SIGNATURES = {
                                   _i32, _vp]),
     "qsa_prefill_intervals": (C.c_int, [_vp, _vp, _vp, _i32, _i64, _vp, _vp, _vp]),
     "qsa_topk": (C.c_int, [_vp, _i64, _vp, _i64, _i32, _i32, _vp, _i64, _vp]),
+    "qsa_topk_ws": (C.c_int, [_vp, _i64, _vp, _i64, _i32, _i32, _vp, _i64, _vp, C.c_size_t, _vp]),
+    "qsa_topk_workspace_size": (C.c_size_t, [_i64, _i32, _i32]),
     "qsa_mqa_prefill_topk": (C.c_int, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _i64, _f32, _i32,
                                        _i32, _vp, _i64, _vp, _sz, _vp]),
     "qsa_prefill_topk_workspace_size": (_sz, [_i64, _i32]),
@@ -221,9 +223,14 @@ def prefill_intervals(cu_seqlens_q: torch.Tensor, seq_lens: torch.Tensor, key_of
     return ks, ke
 
 
+def topk_workspace_size(rows: int, W: int, k: int) -> int:
+    return int(lib().qsa_topk_workspace_size(rows, W, k))
+
+
 def topk(scores: torch.Tensor, k: int, lengths: torch.Tensor | None = None, idx: torch.Tensor | None = None,
-         stream=None) -> torch.Tensor:
-    """Top-k column indices int32 [rows, k] (ascending, -1 padded) of score rows fp32 [rows, W]."""
+         stream=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Top-k column indices int32 [rows, k] (ascending, -1 padded) of score rows fp32 [rows, W];
+    with a workspace (a device tensor of at least topk_workspace_size bytes) through qsa_topk_ws."""
     _need(scores, "scores", torch.float32, 2)
     if scores.stride(1) != 1:
         raise ValueError("scores need a unit column stride")
@@ -237,6 +244,13 @@ def topk(scores: torch.Tensor, k: int, lengths: torch.Tensor | None = None, idx:
     _need(idx, "idx", torch.int32, 2)
     if idx.shape != (rows, k) or idx.stride(1) != 1:
         raise ValueError("idx must be [rows, k] with unit column stride")
+    if workspace is not None:
+        if not workspace.is_contiguous():
+            raise ValueError("workspace must be contiguous")
+        nbytes = workspace.numel() * workspace.element_size()
+        _check("qsa_topk_ws", lib().qsa_topk_ws(_ptr(scores), scores.stride(0), _ptr(lengths), rows, W, k, _ptr(idx),
+                                                idx.stride(0), _ptr(workspace), nbytes, _stream(stream)))
+        return idx
     _check("qsa_topk", lib().qsa_topk(_ptr(scores), scores.stride(0), _ptr(lengths), rows, W, k, _ptr(idx),
                                       idx.stride(0), _stream(stream)))
     return idx

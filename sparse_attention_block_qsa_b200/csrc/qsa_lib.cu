@@ -145,6 +145,8 @@ qsa_status_t device_info(int* sms) {
         {reinterpret_cast<const void*>(qsa::attn::attn_kernel), qsa::attn::SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_rows_kernel), qsa::topk::ROWS_SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_pipe_kernel), qsa::topk::PIPE_SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::topk::topk_filter_kernel), qsa::topk::TP_SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::topk::topk_list_kernel), qsa::topk::TP_LIST_SMEM_BYTES},
     };
     for (auto& k : kernels) {
       e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k.bytes);
@@ -333,7 +335,8 @@ qsa_status_t validate_topk(const TopkArgs& a) {
 constexpr size_t kPredBytes = 4096;
 constexpr int64_t kPredFloats = kPredBytes / sizeof(float);
 
-qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream, float* pred_state = nullptr) {
+qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream, float* pred_state = nullptr,
+                         uint8_t* ws = nullptr) {
   int sms = 0;
   qsa_status_t st = device_info(&sms);
   if (st != QSA_OK) return st;
@@ -348,9 +351,33 @@ qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream, float* pred_sta
   p.vec4 = aligned(a.scores, 16) && (p.stride % 4 == 0);
   p.rows = a.rows;
   p.pred_state = pred_state;
+  p.row_list = nullptr;
+  p.row_count = nullptr;
+  p.ws = ws;
   // the predictions carried between chunks hold one float per CTA
   const int64_t max_grid = pred_state ? kPredFloats : INT32_MAX;
-  if (p.vec4 && a.W % 4 == 0) {
+  if (ws != nullptr && p.vec4 && a.W % 4 == 0) {
+    // with a workspace: filter pass, list selection, exact pass over the rows that missed
+    using namespace qsa::topk;
+    const TpLayout L = tp_layout(a.rows);
+    const int64_t grid_f = std::min<int64_t>(std::min<int64_t>(a.rows, (int64_t)sms * TP_CTAS_PER_SM), TP_PRED_FLOATS);
+    Params f = p;
+    f.pred_state = reinterpret_cast<float*>(ws + L.pred);  // carried between calls through the workspace
+    topk_filter_kernel<<<(unsigned)grid_f, TP_THREADS, TP_SMEM_BYTES, stream>>>(f);
+    st = launch_status("top-k filter kernel");
+    if (st != QSA_OK) return st;
+    const int64_t grid_l = std::min<int64_t>((a.rows + TP_LIST_WARPS - 1) / TP_LIST_WARPS,
+                                             (int64_t)sms * TP_LIST_CTAS_PER_SM);
+    topk_list_kernel<<<(unsigned)grid_l, TP_LIST_WARPS * 32, TP_LIST_SMEM_BYTES, stream>>>(p);
+    st = launch_status("top-k list kernel");
+    if (st != QSA_OK) return st;
+    Params q = p;
+    q.pred_state = nullptr;
+    q.row_list = reinterpret_cast<const int32_t*>(ws + L.list);
+    q.row_count = reinterpret_cast<const uint32_t*>(ws + L.count);
+    topk_rows_kernel<<<(unsigned)std::min<int64_t>(a.rows, (int64_t)sms * ROWS_CTAS_PER_SM), THREADS, ROWS_SMEM_BYTES,
+                       stream>>>(q);
+  } else if (p.vec4 && a.W % 4 == 0) {
     // rows start on 16-byte boundaries: stream them with bulk copies
     const int64_t grid = std::min<int64_t>(std::min<int64_t>(a.rows, (int64_t)sms * qsa::topk::PIPE_CTAS_PER_SM), max_grid);
     qsa::topk::topk_pipe_kernel<<<(unsigned)grid, qsa::topk::PIPE_THREADS, qsa::topk::PIPE_SMEM_BYTES, stream>>>(p);
@@ -651,6 +678,33 @@ qsa_status_t qsa_topk(const float* scores, int64_t score_stride, const int32_t* 
   if (st != QSA_OK) return st;
   if (rows == 0) return ok();
   return launch_topk(a, static_cast<cudaStream_t>(stream));
+}
+
+size_t qsa_topk_workspace_size(int64_t rows, int32_t W, int32_t k) {
+  (void)W;
+  (void)k;
+  return rows > 0 ? qsa::topk::tp_layout(rows).total : 0;
+}
+
+qsa_status_t qsa_topk_ws(const float* scores, int64_t score_stride, const int32_t* lengths, int64_t rows, int32_t W,
+                         int32_t k, int32_t* idx, int64_t idx_stride, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  TopkArgs a{scores, score_stride, lengths, rows, W, k, idx, idx_stride};
+  qsa_status_t st = validate_topk(a);
+  if (st != QSA_OK) return st;
+  if (rows == 0) return ok();
+  const size_t need = qsa_topk_workspace_size(rows, W, k);
+  if (!workspace) return fail(QSA_ERR_INVALID_ARG, "null workspace");
+  if (!aligned(workspace, 256)) return fail(QSA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  if (workspace_bytes < need)
+    return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes; %zu needed for %lld rows", workspace_bytes, need,
+                (long long)rows);
+  const Range rw{reinterpret_cast<uintptr_t>(workspace), reinterpret_cast<uintptr_t>(workspace) + need};
+  if (overlaps(rw, span(scores, 4, rows, rows > 1 ? score_stride : W, 1, 0, 1, 0, W)) ||
+      overlaps(rw, span(idx, 4, rows, rows > 1 ? idx_stride : k, 1, 0, 1, 0, k)) ||
+      (lengths && overlaps(rw, span(lengths, 4, rows, 1, 1, 0, 1, 0, 1))))
+    return fail(QSA_ERR_INVALID_ARG, "workspace overlaps an argument");
+  return launch_topk(a, static_cast<cudaStream_t>(stream), nullptr, static_cast<uint8_t*>(workspace));
 }
 
 qsa_status_t qsa_mqa_prefill_topk_noalloc(const void* q, int64_t q_stride_t, int64_t q_stride_h, const void* k,

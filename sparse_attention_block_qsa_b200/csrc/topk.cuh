@@ -65,6 +65,9 @@ struct Params {
   int64_t idx_stride;
   int32_t vec4;            // rows are 16-byte aligned: use float4 loads
   float* pred_state;       // per-CTA predictions carried between launches (may be null)
+  const int32_t* row_list;    // rows kernel: if set, only these rows (exact path), row_count of them
+  const uint32_t* row_count;
+  uint8_t* ws;                // two-pass kernels: the caller's workspace (tp_layout)
 };
 
 // Order-preserving key of a score; 0 marks "not a candidate".
@@ -588,7 +591,14 @@ __global__ void __launch_bounds__(THREADS, ROWS_CTAS_PER_SM) topk_rows_kernel(co
   float pred = p.pred_state ? p.pred_state[blockIdx.x] : 0.f;
   for (int i = tid; i < BM_WORDS; i += THREADS) S.gt[i] = S.tie[i] = 0;
 
-  for (int64_t r = r_begin; r < r_end; ++r) {
+  // list mode: the rows another pass could not resolve, exact path only
+  const uint32_t n_list = p.row_list ? *(volatile const uint32_t*)p.row_count : 0u;
+  const int64_t i_begin = p.row_list ? blockIdx.x : r_begin;
+  const int64_t i_end = p.row_list ? (int64_t)n_list : r_end;
+  const int64_t i_step = p.row_list ? gridDim.x : 1;
+  if (p.row_list) pred = 0.f;
+  for (int64_t i = i_begin; i < i_end; i += i_step) {
+    const int64_t r = p.row_list ? (int64_t)p.row_list[i] : i;
     const float* row = p.scores + r * p.stride;
     const int len = row_len(p, r);
     start_row(S);
@@ -610,11 +620,11 @@ __global__ void __launch_bounds__(THREADS, ROWS_CTAS_PER_SM) topk_rows_kernel(co
     }
     if (!done) exact_select<BlockSync>(p, S, row, len, false, thr, need_tie);
     __syncthreads();
-    if (!done) pred = next_prediction(thr);  // a miss refreshes the prediction
+    if (!done && !p.row_list) pred = next_prediction(thr);  // a miss refreshes the prediction
     write_row<BlockSync>(p, S, p.idx + r * p.idx_stride, (len + 31) >> 5, need_tie);
     __syncthreads();
   }
-  if (p.pred_state && tid == 0) p.pred_state[blockIdx.x] = pred;
+  if (p.pred_state && !p.row_list && tid == 0) p.pred_state[blockIdx.x] = pred;
 }
 
 constexpr size_t ROWS_SMEM_BYTES = sizeof(Sel);
@@ -887,6 +897,465 @@ __global__ void __launch_bounds__(PIPE_THREADS, PIPE_CTAS_PER_SM) topk_pipe_kern
     ConsumerSync::sync();
   }
   if (p.pred_state && tid == 0) p.pred_state[blockIdx.x] = M.pred_next;
+}
+
+// -------------------------------------------------------------- two-pass kernels (caller workspace)
+//
+// With a workspace (qsa_topk_ws) the aligned-row selection runs in three
+// launches, so that no CTA both streams a row and resolves one:
+//  * topk_filter_kernel (four CTAs per SM): a producer warp streams the rows
+//    as 16 KB bulk copies into a 3-slot ring; 8 filtering warps compare every
+//    score with the prediction, write the candidates (key and column) to the
+//    row's list in the workspace (up to 4096: warp w owns list segment w of
+//    512, positions from a warp scan) and count them in a 256-bin histogram
+//    of key offsets above the prediction (bins of 2^15 key steps: one
+//    binade, the last bin taking everything above).  At the end of a row the
+//    histogram gives the bin of its k-th key, so the prediction for the next
+//    row follows every row: 0.85 x the bin's lower edge, kept unchanged while
+//    it stays within 0.75 .. 0.9 of that edge (a CPU replay of the 4 x
+//    4,096-row workload's rows: 0.4% of rows short of k, almost none over a
+//    segment).  A row without a prediction, with fewer than k candidates or
+//    with a full segment is marked for the exact pass.
+//  * topk_list_kernel: one warp per row, no block barriers: the stored
+//    histogram gives the boundary bin, one pass over the list marks the
+//    columns of higher bins in the warp's column bitmap and sets the boundary
+//    bin's entries aside, the warp ranks those (at most 32, else the row goes
+//    to the exact pass; larger key first, then lower column) and writes the
+//    bitmap out in ascending order.
+//  * topk_rows_kernel in list mode: the exact path over the marked rows.
+
+constexpr int TP_FILT_WARPS = 8;
+constexpr int TP_THREADS = (TP_FILT_WARPS + 1) * 32;
+constexpr int TP_CTAS_PER_SM = 4;
+constexpr int TP_NST = 3;
+constexpr int TP_CAP = 4096;          // staged candidates per row (global memory, so roomier than CAP)
+constexpr int TP_SEG = TP_CAP / TP_FILT_WARPS;
+constexpr int TP_BINS = 256;
+constexpr int TP_SHIFT = 15;
+constexpr float TP_MARGIN = 0.85f;
+constexpr float TP_KEEP_LO = 0.75f;
+constexpr float TP_KEEP_HI = 0.9f;
+constexpr uint32_t TP_FILTER_BAR = 1;
+constexpr int TP_LIST_WARPS = 8;
+constexpr int TP_LIST_CTAS_PER_SM = 3;
+
+struct TpRowHdr {        // one row's staged list (64 bytes)
+  uint32_t cnt[TP_FILT_WARPS];  // entries appended by each filtering warp (may pass TP_SEG)
+  uint32_t kmax;
+  float pred;            // the threshold the row was filtered with
+  uint32_t status;       // 0: the list holds every selected column; 1: exact pass
+  uint32_t pad[5];
+};
+static_assert(sizeof(TpRowHdr) == 64, "row header size");
+
+// Workspace of the two-pass kernels for `rows` rows (offsets multiples of 256 bytes).
+struct TpLayout {
+  size_t hdr, hist, keys, cols, count, list, pred, total;
+};
+constexpr int TP_PRED_FLOATS = 1024;   // per-CTA predictions carried from one call to the next
+__host__ __device__ inline size_t tp_round(size_t x) { return (x + 255) & ~size_t(255); }
+__host__ __device__ inline TpLayout tp_layout(int64_t rows) {
+  TpLayout L;
+  const size_t r = rows > 0 ? (size_t)rows : 0;
+  L.hdr = 0;
+  L.hist = tp_round(L.hdr + r * sizeof(TpRowHdr));
+  L.keys = tp_round(L.hist + r * TP_BINS * 4);
+  L.cols = tp_round(L.keys + r * TP_CAP * 4);
+  L.count = tp_round(L.cols + r * TP_CAP * 2);
+  L.list = tp_round(L.count + 4);
+  L.pred = tp_round(L.list + r * 4);
+  L.total = tp_round(L.pred + TP_PRED_FLOATS * 4);
+  return L;
+}
+
+__device__ __forceinline__ uint32_t tp_bin(uint32_t key, uint32_t key_lo) {
+  return min((key - key_lo) >> TP_SHIFT, (uint32_t)(TP_BINS - 1));
+}
+
+struct TpSmem {
+  float ring[TP_NST * CHUNK];
+  uint64_t full[TP_NST];
+  uint64_t empty[TP_NST];
+  uint32_t hist[TP_BINS];
+  uint32_t cnt[TP_FILT_WARPS];
+  uint32_t kmax;
+  float pred;        // this row's threshold
+  float pred_next;   // the next row's
+  int abort;
+  int stop;
+};
+constexpr size_t TP_SMEM_BYTES = sizeof(TpSmem) + 128;
+
+__global__ void __launch_bounds__(TP_THREADS, TP_CTAS_PER_SM) topk_filter_kernel(const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  TpSmem& M = *reinterpret_cast<TpSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t k = (uint32_t)p.k;
+  const TpLayout L = tp_layout(p.rows);
+  TpRowHdr* hdrs = reinterpret_cast<TpRowHdr*>(p.ws + L.hdr);
+  uint32_t* ghist = reinterpret_cast<uint32_t*>(p.ws + L.hist);
+  uint32_t* gkeys = reinterpret_cast<uint32_t*>(p.ws + L.keys);
+  uint16_t* gcols = reinterpret_cast<uint16_t*>(p.ws + L.cols);
+  const int64_t r_begin = (int64_t)blockIdx.x * p.rows / gridDim.x;
+  const int64_t r_end = (int64_t)(blockIdx.x + 1) * p.rows / gridDim.x;
+
+  if (tid == 0) {
+    for (int s = 0; s < TP_NST; ++s) {
+      mbar_init(&M.full[s], 1);
+      mbar_init(&M.empty[s], TP_FILT_WARPS);
+    }
+    M.abort = 0;
+    // a prediction left in the workspace by an earlier call (any bit pattern:
+    // only the speed depends on it)
+    const float carried = p.pred_state ? p.pred_state[blockIdx.x] : 0.f;
+    M.pred_next = carried > 0.f && carried < 3.0e38f ? carried : 0.f;
+    if (blockIdx.x == 0) *reinterpret_cast<uint32_t*>(p.ws + L.count) = 0u;  // the exact pass's row count
+    fence_mbar_init();
+  }
+  for (int i = tid; i < TP_BINS; i += TP_THREADS) M.hist[i] = 0;
+  __syncthreads();
+
+  if (warp == TP_FILT_WARPS) {
+    // ================= producer: every chunk of every row, back to back
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int64_t r = r_begin; r < r_end && !*(volatile int*)&M.abort; ++r) {
+        const int len4 = (row_len(p, r) + 3) & ~3;  // within the row: W is a multiple of 4
+        const float* row = p.scores + r * p.stride;
+        for (int c0 = 0; c0 < len4; c0 += CHUNK, ++it) {
+          const int s = it % TP_NST;
+          if (!mbar_wait(&M.empty[s], ((it / TP_NST) & 1) ^ 1, &M.abort)) {
+            if (atomicExch(&M.abort, 1) == 0) record_device_error(QSA_DEVERR_WAIT_TIMEOUT);
+            break;
+          }
+          const uint32_t bytes = (uint32_t)min(CHUNK, len4 - c0) * 4u;
+          mbar_arrive_expect_tx(&M.full[s], bytes);
+          asm volatile(
+              "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                  smem_addr(M.ring + s * CHUNK)),
+              "l"(row + c0), "r"(bytes), "r"(smem_addr(&M.full[s]))
+              : "memory");
+        }
+      }
+      // the last copy into every slot must land before the block may retire
+      for (uint32_t i = it > (uint32_t)TP_NST ? it - TP_NST : 0u; i < it; ++i)
+        if (!mbar_wait(&M.full[i % TP_NST], (i / TP_NST) & 1, nullptr)) break;
+    }
+    __syncwarp();
+    return;
+  }
+
+  // ================= 8 filtering warps
+  const int fw = warp;
+  uint32_t it = 0;
+  for (int64_t r = r_begin; r < r_end; ++r) {
+    if (tid == 0) {
+      M.pred = M.pred_next;
+      M.kmax = 0;
+      M.stop = *(volatile int*)&M.abort;
+    }
+    named_barrier_sync(TP_FILTER_BAR, TP_FILT_WARPS * 32);
+    if (M.stop) break;
+    const float pred = M.pred;
+    const bool fast = pred > 0.f;
+    const uint32_t key_lo = __float_as_uint(pred) | 0x80000000u;
+    const int len = row_len(p, r);
+    const int len4 = (len + 3) & ~3;
+    uint32_t* keys = gkeys + r * TP_CAP + fw * TP_SEG;
+    uint16_t* cols = gcols + r * TP_CAP + fw * TP_SEG;
+    uint32_t kmax = 0, count = 0;  // kmax: largest candidate key (every score's without a prediction)
+    for (int c0 = 0; c0 < len4; c0 += CHUNK, ++it) {
+      const int s = it % TP_NST;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&M.full[s], (it / TP_NST) & 1, &M.abort));
+      if (!ok) {
+        if (lane == 0 && atomicExch(&M.abort, 1) == 0) record_device_error(QSA_DEVERR_WAIT_TIMEOUT);
+      } else {
+        const float4* ring4 = reinterpret_cast<const float4*>(M.ring + s * CHUNK);
+        const bool tail = c0 + CHUNK > len;
+        constexpr int U = CHUNK / 4 / (TP_FILT_WARPS * 32);  // float4 per thread per chunk
+        uint32_t mask = 0;  // bit 4u + e: score e of this lane's u-th float4 is a candidate
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int f = u * TP_FILT_WARPS * 32 + tid;
+          float4 x = ring4[f];
+          const int j0 = c0 + 4 * f;
+          if (tail) {
+            if (j0 >= len) x.x = -INFINITY;
+            if (j0 + 1 >= len) x.y = -INFINITY;
+            if (j0 + 2 >= len) x.z = -INFINITY;
+            if (j0 + 3 >= len) x.w = -INFINITY;
+          }
+          if (fast) {
+            mask |= (uint32_t)(x.x >= pred) << (4 * u) | (uint32_t)(x.y >= pred) << (4 * u + 1) |
+                    (uint32_t)(x.z >= pred) << (4 * u + 2) | (uint32_t)(x.w >= pred) << (4 * u + 3);
+          } else {
+            kmax = max(kmax, max(max(score_key(x.x), score_key(x.y)), max(score_key(x.z), score_key(x.w))));
+          }
+        }
+        if (fast) {
+          const uint32_t nl = __popc(mask);
+          uint32_t incl = nl;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          uint32_t pos = count + incl - nl;
+          count += __shfl_sync(0xffffffffu, incl, 31);
+          while (mask) {
+            const int b = __ffs(mask) - 1;
+            mask &= mask - 1;
+            const int f = (b >> 2) * TP_FILT_WARPS * 32 + tid;
+            const float x = M.ring[s * CHUNK + 4 * f + (b & 3)];
+            const uint32_t key = __float_as_uint(x) | 0x80000000u;  // x >= pred > 0
+            atomicAdd(&M.hist[tp_bin(key, key_lo)], 1u);
+            if (pos < (uint32_t)TP_SEG) {
+              keys[pos] = key;
+              cols[pos] = (uint16_t)(c0 + 4 * f + (b & 3));
+            }
+            kmax = max(kmax, key);
+            ++pos;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&M.empty[s]);
+    }
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+      M.cnt[fw] = count;
+      atomicMax(&M.kmax, kmax);
+    }
+    named_barrier_sync(TP_FILTER_BAR, TP_FILT_WARPS * 32);
+    // ---- end of the row: header, histogram, the next row's prediction
+    uint32_t n = 0;
+    bool overflow = false;
+#pragma unroll
+    for (int w = 0; w < TP_FILT_WARPS; ++w) {
+      n += M.cnt[w];
+      overflow |= M.cnt[w] > (uint32_t)TP_SEG;
+    }
+    const bool exact = !fast || n < k || overflow;
+    ghist[r * TP_BINS + tid] = M.hist[tid];
+    if (warp == 0) {
+      float next = M.pred_next;
+      if (!fast) {
+        const uint32_t km = M.kmax;  // the row's largest score: a first guess
+        next = (km & 0x80000000u) && key_value(km) > 0.f ? 0.5f * key_value(km) : 0.f;
+      } else if (n < k) {
+        next = 2 * n >= k ? pred * 0.8f : 0.f;  // far too high (a stale carried value): start over from the max
+      } else {
+        // the bin holding the k-th candidate (lane l: bins 255 - 8l .. 248 - 8l)
+        uint32_t c[TP_BINS / 32], sum = 0;
+#pragma unroll
+        for (int b = 0; b < TP_BINS / 32; ++b) {
+          c[b] = M.hist[TP_BINS - 1 - (TP_BINS / 32) * lane - b];
+          sum += c[b];
+        }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - sum;
+        uint32_t bsel = 0, acc = excl;
+        bool found = false;
+#pragma unroll
+        for (int b = 0; b < TP_BINS / 32; ++b) {
+          const bool here = !found && acc + c[b] >= k;
+          if (here) bsel = TP_BINS - 1 - (TP_BINS / 32) * lane - b;
+          if (!found && !here) acc += c[b];
+          found = found || here;
+        }
+        const unsigned who = __ballot_sync(0xffffffffu, excl < k && k <= incl);
+        bsel = __shfl_sync(0xffffffffu, bsel, who ? __ffs(who) - 1 : 0);
+        if (bsel == (uint32_t)(TP_BINS - 1)) {
+          next = pred * 1.5f;  // the k-th key lies a binade or more above the threshold
+        } else {
+          const float edge = key_value(key_lo + (bsel << TP_SHIFT));
+          if (!(pred >= TP_KEEP_LO * edge && pred <= TP_KEEP_HI * edge)) next = TP_MARGIN * edge;
+        }
+      }
+      if (lane == 0) {
+        M.pred_next = next;
+        TpRowHdr h;
+#pragma unroll
+        for (int w = 0; w < TP_FILT_WARPS; ++w) h.cnt[w] = M.cnt[w];
+        h.kmax = M.kmax;
+        h.pred = pred;
+        h.status = exact ? 1u : 0u;
+#pragma unroll
+        for (int i = 0; i < 5; ++i) h.pad[i] = 0;
+        hdrs[r] = h;
+      }
+    }
+    named_barrier_sync(TP_FILTER_BAR, TP_FILT_WARPS * 32);
+    M.hist[tid] = 0;  // the next row's histogram (appends begin after the next barrier)
+  }
+  if (p.pred_state && tid == 0) p.pred_state[blockIdx.x] = M.pred_next;
+}
+
+struct TpListWarp {
+  uint32_t bm[BM_WORDS];   // selected columns of the current row
+  uint32_t small_key[32];
+  int32_t small_col[32];
+  uint32_t n_small;
+  uint32_t pad[31];
+};
+constexpr size_t TP_LIST_SMEM_BYTES = TP_LIST_WARPS * sizeof(TpListWarp);
+
+__global__ void __launch_bounds__(TP_LIST_WARPS * 32, TP_LIST_CTAS_PER_SM) topk_list_kernel(const Params p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  TpListWarp& S = reinterpret_cast<TpListWarp*>(smem_raw)[warp];
+  const uint32_t k = (uint32_t)p.k;
+  const TpLayout L = tp_layout(p.rows);
+  const TpRowHdr* hdrs = reinterpret_cast<const TpRowHdr*>(p.ws + L.hdr);
+  const uint32_t* ghist = reinterpret_cast<const uint32_t*>(p.ws + L.hist);
+  const uint32_t* gkeys = reinterpret_cast<const uint32_t*>(p.ws + L.keys);
+  const uint16_t* gcols = reinterpret_cast<const uint16_t*>(p.ws + L.cols);
+  uint32_t* miss_count = reinterpret_cast<uint32_t*>(p.ws + L.count);
+  int32_t* miss_rows = reinterpret_cast<int32_t*>(p.ws + L.list);
+  for (int i = lane; i < BM_WORDS; i += 32) S.bm[i] = 0;
+  if (lane == 0) S.n_small = 0;
+  __syncwarp();
+  const int64_t nw = (int64_t)gridDim.x * TP_LIST_WARPS;
+  for (int64_t r = (int64_t)blockIdx.x * TP_LIST_WARPS + warp; r < p.rows; r += nw) {
+    const TpRowHdr& h = hdrs[r];
+    const uint32_t status = h.status;
+    uint32_t B = 0, needB = 0;
+    bool exact = status != 0u;
+    if (!exact) {
+      // the bin of the k-th candidate and how many of its entries to take
+      uint32_t c[TP_BINS / 32], sum = 0;
+#pragma unroll
+      for (int b = 0; b < TP_BINS / 32; ++b) {
+        c[b] = ghist[r * TP_BINS + TP_BINS - 1 - (TP_BINS / 32) * lane - b];
+        sum += c[b];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - sum;
+      uint32_t bsel = 0, acc = excl, csel = 0;
+      bool found = false;
+#pragma unroll
+      for (int b = 0; b < TP_BINS / 32; ++b) {
+        const bool here = !found && acc + c[b] >= k;
+        if (here) {
+          bsel = TP_BINS - 1 - (TP_BINS / 32) * lane - b;
+          csel = c[b];
+        }
+        if (!found && !here) acc += c[b];
+        found = found || here;
+      }
+      const unsigned who = __ballot_sync(0xffffffffu, excl < k && k <= incl);
+      const int src = who ? __ffs(who) - 1 : 0;
+      B = __shfl_sync(0xffffffffu, bsel, src);
+      needB = k - __shfl_sync(0xffffffffu, acc, src);
+      const uint32_t nb = __shfl_sync(0xffffffffu, csel, src);
+      exact = who == 0u || B == (uint32_t)(TP_BINS - 1) || nb > 32u;
+    }
+    if (exact) {
+      if (lane == 0) miss_rows[atomicAdd(miss_count, 1u)] = (int32_t)r;
+      continue;
+    }
+    const uint32_t key_lo = __float_as_uint(h.pred) | 0x80000000u;
+    // one pass over the list: higher bins are taken, the boundary bin is set
+    // aside.  Entry e of the row (segments back to back) is slot e - pre[s]
+    // of segment s; each lane loads TP_BATCH entries before using any.
+    const uint32_t my_cnt = lane < TP_FILT_WARPS ? min(h.cnt[lane], (uint32_t)TP_SEG) : 0u;
+    uint32_t pre_incl = my_cnt;
+#pragma unroll
+    for (int o = 1; o < TP_FILT_WARPS; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, pre_incl, o);
+      if (lane >= o) pre_incl += y;
+    }
+    const uint32_t n_all = __shfl_sync(0xffffffffu, pre_incl, TP_FILT_WARPS - 1);
+    const uint32_t pre_excl = pre_incl - my_cnt;
+    uint32_t first[TP_FILT_WARPS];  // first entry of each segment
+#pragma unroll
+    for (int sgm = 0; sgm < TP_FILT_WARPS; ++sgm) first[sgm] = __shfl_sync(0xffffffffu, pre_excl, sgm);
+    const uint32_t* rkeys = gkeys + r * TP_CAP;
+    const uint16_t* rcols = gcols + r * TP_CAP;
+    constexpr int TP_BATCH = 8;
+    for (uint32_t e0 = 0; e0 < n_all; e0 += 32 * TP_BATCH) {
+      uint32_t key[TP_BATCH];
+      int col[TP_BATCH];
+#pragma unroll
+      for (int u = 0; u < TP_BATCH; ++u) {
+        const uint32_t e = e0 + u * 32 + lane;
+        // segment of entry e: the last segment whose first entry is <= e
+        uint32_t slot = 0;
+#pragma unroll
+        for (int sgm = 0; sgm < TP_FILT_WARPS; ++sgm)
+          if (e >= first[sgm]) slot = (uint32_t)sgm * TP_SEG + (e - first[sgm]);
+        key[u] = e < n_all ? __ldg(rkeys + slot) : 0u;
+        col[u] = e < n_all ? (int)__ldg(rcols + slot) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < TP_BATCH; ++u) {
+        if (e0 + u * 32 + lane < n_all) {
+          const uint32_t b = tp_bin(key[u], key_lo);
+          const int j = col[u];
+          if (b > B) {
+            atomicOr(&S.bm[j >> 5], 1u << (j & 31));
+          } else if (b == B) {
+            const uint32_t q = atomicAdd(&S.n_small, 1u);
+            S.small_key[q] = key[u];
+            S.small_col[q] = j;
+          }
+        }
+      }
+    }
+    __syncwarp();
+    {
+      // rank the boundary entries: larger key first, then lower column
+      const uint32_t nb = S.n_small;
+      const bool have = (uint32_t)lane < nb;
+      const uint32_t key = have ? S.small_key[lane] : 0u;
+      const int32_t j = have ? S.small_col[lane] : INT32_MAX;
+      uint32_t rank = 0;
+      for (uint32_t o = 0; o < nb; ++o) {
+        const uint32_t ko = S.small_key[o];
+        const int32_t jo = S.small_col[o];
+        rank += (ko > key) || (ko == key && jo < j);
+      }
+      if (have && rank < needB) atomicOr(&S.bm[j >> 5], 1u << (j & 31));
+    }
+    __syncwarp();
+    if (lane == 0) S.n_small = 0;
+    // the bitmap out in ascending order (exactly k bits are set); words cleared on the way
+    const int len = row_len(p, r);
+    const int nwords = (len + 31) >> 5;
+    const int wpl = (nwords + 31) >> 5;
+    const int w0 = min(lane * wpl, nwords), w1 = min(w0 + wpl, nwords);
+    uint32_t cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += (uint32_t)__popc(S.bm[w]);
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    uint32_t pos = incl - cnt;
+    int32_t* out = p.idx + r * p.idx_stride;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = S.bm[w];
+      S.bm[w] = 0;
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (pos < k) out[pos] = w * 32 + b;
+        ++pos;
+      }
+    }
+    __syncwarp();
+  }
 }
 
 }  // namespace topk

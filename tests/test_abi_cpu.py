@@ -161,6 +161,38 @@ def test_topk_rejects(kw, code):
     assert st == code, detail
 
 
+def topk_ws(ws=None, nbytes=None, **kw):
+    a = dict(s=A, ss=5000, ln=0, rows=10, W=5000, k=512, idx=A + S, iss=512)
+    a.update(kw)
+    L = qsa.lib()
+    need = L.qsa_topk_workspace_size(a["rows"], a["W"], a["k"])
+    ws = A + 2 * S if ws is None else ws
+    nbytes = need if nbytes is None else nbytes
+    st = L.qsa_topk_ws(a["s"], a["ss"], a["ln"] or None, a["rows"], a["W"], a["k"], a["idx"], a["iss"], ws, nbytes,
+                       None)
+    return st, L.qsa_last_error_detail().decode()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=0), UNSUP), (dict(rows=-1), INVALID), (dict(s=A + 2), ALIGN),
+    (dict(ws=0), INVALID), (dict(ws=A + 2 * S + 128), ALIGN), (dict(nbytes=1000), WS),
+    (dict(ws=A), INVALID),                              # the workspace overlaps scores
+    (dict(ws=A + S - 256), INVALID),                    # ... and idx
+])
+def test_topk_ws_rejects(kw, code):
+    st, detail = topk_ws(**kw)
+    assert st == code, detail
+
+
+def test_topk_workspace_size():
+    L = qsa.lib()
+    size = L.qsa_topk_workspace_size
+    # per row: a 64-byte header, a 256-bin histogram, 4096 keys and 4096 columns
+    assert size(16384, 26624, 512) >= 16384 * (64 + 1024 + 4096 * 6)
+    assert size(1, 26624, 512) < size(2, 26624, 512) and size(0, 100, 5) == 0
+    assert size(1000, 100, 5) % 256 == 0
+
+
 def test_fused_rejects_small_workspace():
     L = qsa.lib()
     st = L.qsa_mqa_prefill_topk(A, 512, 128, A + S, 128, 1000, A + 2 * S, A + 3 * S, 1000, 0.088, 1000, 512,

@@ -17,10 +17,16 @@ SCALE = 1.0 / np.sqrt(128.0)
 DEV = torch.device("cuda")
 
 
-def gpu_topk(scores: np.ndarray, k: int, lengths=None):
+def gpu_topk(scores: np.ndarray, k: int, lengths=None, ws: bool = False):
+    """qsa_topk, or with ws the workspace path (filter pass, list selection,
+    exact pass) over the same rows."""
     s = torch.from_numpy(scores.astype(np.float32)).to(DEV)
     ln = None if lengths is None else torch.from_numpy(lengths.astype(np.int32)).to(DEV)
-    idx = qsa.topk(s, k, lengths=ln)
+    workspace = None
+    if ws:
+        n = qsa.topk_workspace_size(s.shape[0], s.shape[1], k)
+        workspace = torch.full((n,), 0x5A, dtype=torch.uint8, device=DEV)   # stale contents must not matter
+    idx = qsa.topk(s, k, lengths=ln, workspace=workspace)
     torch.cuda.synchronize()
     assert qsa.device_error() == 0
     return idx.cpu().numpy()
@@ -32,20 +38,22 @@ def ora_topk(scores: np.ndarray, k: int, lengths=None):
     return oracle.topk(s32, np.minimum(np.maximum(ln, 0), s32.shape[1]), k)
 
 
+@pytest.mark.parametrize("ws", [False, True])
 @pytest.mark.parametrize("k", [1, 7, 512, 2048])
 @pytest.mark.parametrize("W", [100, 5000, 26624])
-def test_topk_random_rows(k, W):
+def test_topk_random_rows(k, W, ws):
     rng = np.random.default_rng(k * 7 + W)
     rows = 64
     s = np.abs(rng.normal(size=(rows, W))) * 3
     s[rng.random(size=s.shape) < 0.03] = -np.inf
     lengths = rng.integers(-5, W + 10, size=rows).astype(np.int32)
-    assert np.array_equal(gpu_topk(s, k, lengths), ora_topk(s, k, lengths))
-    assert np.array_equal(gpu_topk(s, k), ora_topk(s, k))
+    assert np.array_equal(gpu_topk(s, k, lengths, ws), ora_topk(s, k, lengths))
+    assert np.array_equal(gpu_topk(s, k, ws=ws), ora_topk(s, k))
 
 
+@pytest.mark.parametrize("ws", [False, True])
 @pytest.mark.parametrize("W,k,rows", [(2048, 256, 9000), (26624, 512, 2400)])
-def test_topk_predictions_across_rows(W, k, rows):
+def test_topk_predictions_across_rows(W, k, rows, ws):
     """Enough rows that each selecting warp takes several in turn, so the
     threshold predicted from one row meets the next: rows whose scale drops
     (the prediction admits fewer than k), jumps (the candidate list
@@ -66,10 +74,11 @@ def test_topk_predictions_across_rows(W, k, rows):
     lengths = np.full(rows, W, dtype=np.int32)
     short = r % 23 == 4
     lengths[short] = rng.integers(0, k + 5, size=int(short.sum()))
-    assert np.array_equal(gpu_topk(s, k, lengths), ora_topk(s, k, lengths))
+    assert np.array_equal(gpu_topk(s, k, lengths, ws), ora_topk(s, k, lengths))
 
 
-def test_topk_ties_signed_zero_negative_and_nan():
+@pytest.mark.parametrize("ws", [False, True])
+def test_topk_ties_signed_zero_negative_and_nan(ws):
     rng = np.random.default_rng(1)
     W, k = 3000, 300
     s = np.round(rng.normal(size=(40, W)), 1)          # heavy ties
@@ -82,13 +91,15 @@ def test_topk_ties_signed_zero_negative_and_nan():
     s[4, rng.random(W) < 0.5] = np.nan                  # NaN never selected
     s[5, :] = np.float32(3.4e38)
     want = ora_topk(np.where(np.isnan(s), -np.inf, s), k)
-    assert np.array_equal(gpu_topk(s, k), want)
+    assert np.array_equal(gpu_topk(s, k, ws=ws), want)
 
 
 def test_topk_uncached_wide_rows_and_odd_stride():
     rng = np.random.default_rng(2)
     s = rng.normal(size=(6, 60000))                     # wider than the shared-memory row cache
     assert np.array_equal(gpu_topk(s, 512), ora_topk(s, 512))
+    s = np.abs(rng.normal(size=(1500, 65536))).astype(np.float32)   # the widest rows, many per CTA
+    assert np.array_equal(gpu_topk(s, 512, ws=True), ora_topk(s, 512))
     # rows that are not 16-byte aligned: scalar loads
     base = torch.from_numpy(rng.normal(size=(20, 1001)).astype(np.float32)).to(DEV)
     view = base[:, 1:]
@@ -160,3 +171,23 @@ def test_fused_prefill_topk_ties_and_skew(sampled_high):
     k[sampled, 0] = 8.0 if sampled_high else 0.0
     k[sampled, 1:] = 0.0
     _fused_vs_separate(p, q, k)
+
+
+def test_topk_workspace_path_matches_streaming_path_at_full_size():
+    """The 4 x 4,096-row, 102,400-token-prefix workload's 16,384 score rows
+    (26,624 columns each, from the prefill kernel): the workspace path and
+    qsa_topk select exactly the same columns (both are exact selections of
+    the same fp32 rows, and every row of the sampled full-parity test checks
+    qsa_topk against the oracle)."""
+    p = wl.make_config(5)
+    ks, ke = oracle.prefill_intervals(p.cu_seqlens_q, p.seq_lens, p.key_offsets)
+    scores = qsa.mqa_prefill(p.q.to(DEV), p.k.to(DEV), torch.from_numpy(ks).to(DEV), torch.from_numpy(ke).to(DEV), p.W)
+    want = qsa.topk(scores, wl.TOPK_K)
+    ws = torch.empty(qsa.topk_workspace_size(p.T, p.W, wl.TOPK_K), dtype=torch.uint8, device=DEV)
+    got = qsa.topk(scores, wl.TOPK_K, workspace=ws)
+    torch.cuda.synchronize()
+    assert qsa.device_error() == 0
+    assert torch.equal(got, want)
+    # a second call over the same workspace (stale lists from the first)
+    got2 = qsa.topk(scores, wl.TOPK_K, workspace=ws)
+    assert torch.equal(got2, want)

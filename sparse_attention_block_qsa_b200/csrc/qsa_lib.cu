@@ -146,7 +146,8 @@ qsa_status_t device_info(int* sms) {
         {reinterpret_cast<const void*>(qsa::topk::topk_rows_kernel), qsa::topk::ROWS_SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_pipe_kernel), qsa::topk::PIPE_SMEM_BYTES},
         {reinterpret_cast<const void*>(qsa::topk::topk_filter_kernel), qsa::topk::TP_SMEM_BYTES},
-        {reinterpret_cast<const void*>(qsa::topk::topk_list_kernel), qsa::topk::TP_LIST_SMEM_BYTES},
+        {reinterpret_cast<const void*>(qsa::topk::topk_list_kernel),
+         qsa::topk::TP_LIST_WARPS * qsa::topk::tp_list_warp_bytes(qsa::topk::MAX_W)},
     };
     for (auto& k : kernels) {
       e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k.bytes);
@@ -368,7 +369,7 @@ qsa_status_t launch_topk(const TopkArgs& a, cudaStream_t stream, float* pred_sta
     if (st != QSA_OK) return st;
     const int64_t grid_l = std::min<int64_t>((a.rows + TP_LIST_WARPS - 1) / TP_LIST_WARPS,
                                              (int64_t)sms * TP_LIST_CTAS_PER_SM);
-    topk_list_kernel<<<(unsigned)grid_l, TP_LIST_WARPS * 32, TP_LIST_SMEM_BYTES, stream>>>(p);
+    topk_list_kernel<<<(unsigned)grid_l, TP_LIST_WARPS * 32, TP_LIST_WARPS * tp_list_warp_bytes(a.W), stream>>>(p);
     st = launch_status("top-k list kernel");
     if (st != QSA_OK) return st;
     Params q = p;

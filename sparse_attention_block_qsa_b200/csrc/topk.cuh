@@ -32,6 +32,8 @@
 // does not depend on the prediction, only the speed does.
 #pragma once
 
+#include <cstddef>
+
 #include "sm100.cuh"
 
 namespace qsa {
@@ -937,7 +939,7 @@ constexpr float TP_KEEP_LO = 0.75f;
 constexpr float TP_KEEP_HI = 0.9f;
 constexpr uint32_t TP_FILTER_BAR = 1;
 constexpr int TP_LIST_WARPS = 8;
-constexpr int TP_LIST_CTAS_PER_SM = 3;
+constexpr int TP_LIST_CTAS_PER_SM = 4;
 
 struct TpRowHdr {        // one row's staged list (64 bytes)
   uint32_t cnt[TP_FILT_WARPS];  // entries appended by each filtering warp (may pass TP_SEG)
@@ -950,7 +952,7 @@ static_assert(sizeof(TpRowHdr) == 64, "row header size");
 
 // Workspace of the two-pass kernels for `rows` rows (offsets multiples of 256 bytes).
 struct TpLayout {
-  size_t hdr, hist, keys, cols, count, list, pred, total;
+  size_t hdr, hist, ent, count, list, pred, total;
 };
 constexpr int TP_PRED_FLOATS = 1024;   // per-CTA predictions carried from one call to the next
 __host__ __device__ inline size_t tp_round(size_t x) { return (x + 255) & ~size_t(255); }
@@ -959,9 +961,8 @@ __host__ __device__ inline TpLayout tp_layout(int64_t rows) {
   const size_t r = rows > 0 ? (size_t)rows : 0;
   L.hdr = 0;
   L.hist = tp_round(L.hdr + r * sizeof(TpRowHdr));
-  L.keys = tp_round(L.hist + r * TP_BINS * 4);
-  L.cols = tp_round(L.keys + r * TP_CAP * 4);
-  L.count = tp_round(L.cols + r * TP_CAP * 2);
+  L.ent = tp_round(L.hist + r * TP_BINS * 4);   // uint2 {key, column} per staged candidate
+  L.count = tp_round(L.ent + r * TP_CAP * 8);
   L.list = tp_round(L.count + 4);
   L.pred = tp_round(L.list + r * 4);
   L.total = tp_round(L.pred + TP_PRED_FLOATS * 4);
@@ -994,8 +995,7 @@ __global__ void __launch_bounds__(TP_THREADS, TP_CTAS_PER_SM) topk_filter_kernel
   const TpLayout L = tp_layout(p.rows);
   TpRowHdr* hdrs = reinterpret_cast<TpRowHdr*>(p.ws + L.hdr);
   uint32_t* ghist = reinterpret_cast<uint32_t*>(p.ws + L.hist);
-  uint32_t* gkeys = reinterpret_cast<uint32_t*>(p.ws + L.keys);
-  uint16_t* gcols = reinterpret_cast<uint16_t*>(p.ws + L.cols);
+  uint2* gent = reinterpret_cast<uint2*>(p.ws + L.ent);
   const int64_t r_begin = (int64_t)blockIdx.x * p.rows / gridDim.x;
   const int64_t r_end = (int64_t)(blockIdx.x + 1) * p.rows / gridDim.x;
 
@@ -1061,8 +1061,7 @@ __global__ void __launch_bounds__(TP_THREADS, TP_CTAS_PER_SM) topk_filter_kernel
     const uint32_t key_lo = __float_as_uint(pred) | 0x80000000u;
     const int len = row_len(p, r);
     const int len4 = (len + 3) & ~3;
-    uint32_t* keys = gkeys + r * TP_CAP + fw * TP_SEG;
-    uint16_t* cols = gcols + r * TP_CAP + fw * TP_SEG;
+    uint2* ent = gent + r * TP_CAP + fw * TP_SEG;
     uint32_t kmax = 0, count = 0;  // kmax: largest candidate key (every score's without a prediction)
     for (int c0 = 0; c0 < len4; c0 += CHUNK, ++it) {
       const int s = it % TP_NST;
@@ -1109,10 +1108,7 @@ __global__ void __launch_bounds__(TP_THREADS, TP_CTAS_PER_SM) topk_filter_kernel
             const float x = M.ring[s * CHUNK + 4 * f + (b & 3)];
             const uint32_t key = __float_as_uint(x) | 0x80000000u;  // x >= pred > 0
             atomicAdd(&M.hist[tp_bin(key, key_lo)], 1u);
-            if (pos < (uint32_t)TP_SEG) {
-              keys[pos] = key;
-              cols[pos] = (uint16_t)(c0 + 4 * f + (b & 3));
-            }
+            if (pos < (uint32_t)TP_SEG) ent[pos] = make_uint2(key, (uint32_t)(c0 + 4 * f + (b & 3)));
             kmax = max(kmax, key);
             ++pos;
           }
@@ -1196,28 +1192,33 @@ __global__ void __launch_bounds__(TP_THREADS, TP_CTAS_PER_SM) topk_filter_kernel
   if (p.pred_state && tid == 0) p.pred_state[blockIdx.x] = M.pred_next;
 }
 
+// Per-warp shared memory of the list kernel: the small buffers, then a column
+// bitmap of tp_bitmap_words(W) words.
 struct TpListWarp {
-  uint32_t bm[BM_WORDS];   // selected columns of the current row
   uint32_t small_key[32];
   int32_t small_col[32];
   uint32_t n_small;
-  uint32_t pad[31];
+  uint32_t pad[3];
+  uint32_t bm[1];          // tp_bitmap_words(W) words
 };
-constexpr size_t TP_LIST_SMEM_BYTES = TP_LIST_WARPS * sizeof(TpListWarp);
+__host__ __device__ inline int tp_bitmap_words(int W) { return (((W + 31) >> 5) + 3) & ~3; }
+__host__ __device__ inline size_t tp_list_warp_bytes(int W) {
+  return offsetof(TpListWarp, bm) + (size_t)tp_bitmap_words(W) * 4;
+}
 
 __global__ void __launch_bounds__(TP_LIST_WARPS * 32, TP_LIST_CTAS_PER_SM) topk_list_kernel(const Params p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  TpListWarp& S = reinterpret_cast<TpListWarp*>(smem_raw)[warp];
+  TpListWarp& S = *reinterpret_cast<TpListWarp*>(smem_raw + (size_t)warp * tp_list_warp_bytes(p.W));
+  const int bmw = tp_bitmap_words(p.W);
   const uint32_t k = (uint32_t)p.k;
   const TpLayout L = tp_layout(p.rows);
   const TpRowHdr* hdrs = reinterpret_cast<const TpRowHdr*>(p.ws + L.hdr);
   const uint32_t* ghist = reinterpret_cast<const uint32_t*>(p.ws + L.hist);
-  const uint32_t* gkeys = reinterpret_cast<const uint32_t*>(p.ws + L.keys);
-  const uint16_t* gcols = reinterpret_cast<const uint16_t*>(p.ws + L.cols);
+  const uint2* gent = reinterpret_cast<const uint2*>(p.ws + L.ent);
   uint32_t* miss_count = reinterpret_cast<uint32_t*>(p.ws + L.count);
   int32_t* miss_rows = reinterpret_cast<int32_t*>(p.ws + L.list);
-  for (int i = lane; i < BM_WORDS; i += 32) S.bm[i] = 0;
+  for (int i = lane; i < bmw; i += 32) S.bm[i] = 0;
   if (lane == 0) S.n_small = 0;
   __syncwarp();
   const int64_t nw = (int64_t)gridDim.x * TP_LIST_WARPS;
@@ -1280,8 +1281,7 @@ __global__ void __launch_bounds__(TP_LIST_WARPS * 32, TP_LIST_CTAS_PER_SM) topk_
     uint32_t first[TP_FILT_WARPS];  // first entry of each segment
 #pragma unroll
     for (int sgm = 0; sgm < TP_FILT_WARPS; ++sgm) first[sgm] = __shfl_sync(0xffffffffu, pre_excl, sgm);
-    const uint32_t* rkeys = gkeys + r * TP_CAP;
-    const uint16_t* rcols = gcols + r * TP_CAP;
+    const uint2* rent = gent + r * TP_CAP;
     constexpr int TP_BATCH = 8;
     for (uint32_t e0 = 0; e0 < n_all; e0 += 32 * TP_BATCH) {
       uint32_t key[TP_BATCH];
@@ -1294,8 +1294,9 @@ __global__ void __launch_bounds__(TP_LIST_WARPS * 32, TP_LIST_CTAS_PER_SM) topk_
 #pragma unroll
         for (int sgm = 0; sgm < TP_FILT_WARPS; ++sgm)
           if (e >= first[sgm]) slot = (uint32_t)sgm * TP_SEG + (e - first[sgm]);
-        key[u] = e < n_all ? __ldg(rkeys + slot) : 0u;
-        col[u] = e < n_all ? (int)__ldg(rcols + slot) : 0;
+        const uint2 v = e < n_all ? __ldg(rent + slot) : make_uint2(0u, 0u);
+        key[u] = v.x;
+        col[u] = (int)v.y;
       }
 #pragma unroll
       for (int u = 0; u < TP_BATCH; ++u) {

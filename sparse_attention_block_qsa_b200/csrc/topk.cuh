@@ -1223,18 +1223,21 @@ __global__ void __launch_bounds__(TP_LIST_WARPS * 32, TP_LIST_CTAS_PER_SM) topk_
   __syncwarp();
   const int64_t nw = (int64_t)gridDim.x * TP_LIST_WARPS;
   for (int64_t r = (int64_t)blockIdx.x * TP_LIST_WARPS + warp; r < p.rows; r += nw) {
-    const TpRowHdr& h = hdrs[r];
-    const uint32_t status = h.status;
+    // the row's header and histogram in one round trip
+    const TpRowHdr* h = hdrs + r;
+    const uint32_t status = __ldg(&h->status);
+    const float hpred = __ldg(&h->pred);
+    const uint32_t cnt_l = lane < TP_FILT_WARPS ? __ldg(&h->cnt[lane]) : 0u;
+    uint32_t c[TP_BINS / 32];
+#pragma unroll
+    for (int b = 0; b < TP_BINS / 32; ++b) c[b] = __ldg(ghist + r * TP_BINS + TP_BINS - 1 - (TP_BINS / 32) * lane - b);
     uint32_t B = 0, needB = 0;
     bool exact = status != 0u;
     if (!exact) {
       // the bin of the k-th candidate and how many of its entries to take
-      uint32_t c[TP_BINS / 32], sum = 0;
+      uint32_t sum = 0;
 #pragma unroll
-      for (int b = 0; b < TP_BINS / 32; ++b) {
-        c[b] = ghist[r * TP_BINS + TP_BINS - 1 - (TP_BINS / 32) * lane - b];
-        sum += c[b];
-      }
+      for (int b = 0; b < TP_BINS / 32; ++b) sum += c[b];
       uint32_t incl = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -1265,11 +1268,11 @@ __global__ void __launch_bounds__(TP_LIST_WARPS * 32, TP_LIST_CTAS_PER_SM) topk_
       if (lane == 0) miss_rows[atomicAdd(miss_count, 1u)] = (int32_t)r;
       continue;
     }
-    const uint32_t key_lo = __float_as_uint(h.pred) | 0x80000000u;
+    const uint32_t key_lo = __float_as_uint(hpred) | 0x80000000u;
     // one pass over the list: higher bins are taken, the boundary bin is set
     // aside.  Entry e of the row (segments back to back) is slot e - pre[s]
     // of segment s; each lane loads TP_BATCH entries before using any.
-    const uint32_t my_cnt = lane < TP_FILT_WARPS ? min(h.cnt[lane], (uint32_t)TP_SEG) : 0u;
+    const uint32_t my_cnt = min(cnt_l, (uint32_t)TP_SEG);
     uint32_t pre_incl = my_cnt;
 #pragma unroll
     for (int o = 1; o < TP_FILT_WARPS; o <<= 1) {
@@ -1282,7 +1285,7 @@ __global__ void __launch_bounds__(TP_LIST_WARPS * 32, TP_LIST_CTAS_PER_SM) topk_
 #pragma unroll
     for (int sgm = 0; sgm < TP_FILT_WARPS; ++sgm) first[sgm] = __shfl_sync(0xffffffffu, pre_excl, sgm);
     const uint2* rent = gent + r * TP_CAP;
-    constexpr int TP_BATCH = 8;
+    constexpr int TP_BATCH = 16;
     for (uint32_t e0 = 0; e0 < n_all; e0 += 32 * TP_BATCH) {
       uint32_t key[TP_BATCH];
       int col[TP_BATCH];

@@ -250,9 +250,12 @@ qsa_status_t qsa_topk(const float* scores, int64_t score_stride, const int32_t* 
  *                    threshold predictions along, which only speeds the next
  *                    call up.  Contents on return are undefined.
  *   workspace_bytes  its size.
- * Other arguments as for qsa_topk.  QSA_ERR_WORKSPACE when workspace_bytes
- * is too small; rows whose start is not 16-byte aligned, or W not a multiple
- * of 4, run as in qsa_topk (the workspace is then unused).
+ * Other arguments as for qsa_topk, checked the same way; then
+ * QSA_ERR_INVALID_ARG for a null workspace or one that overlaps an argument,
+ * QSA_ERR_ALIGNMENT when it is not 256-byte aligned, QSA_ERR_WORKSPACE when
+ * workspace_bytes is too small; nothing is launched on an error.  Rows whose
+ * start is not 16-byte aligned, or W not a multiple of 4, run as in qsa_topk
+ * (the workspace is then unused).
  */
 qsa_status_t qsa_topk_ws(const float* scores, int64_t score_stride, const int32_t* lengths, int64_t rows,
                          int32_t W, int32_t k, int32_t* idx, int64_t idx_stride, void* workspace,

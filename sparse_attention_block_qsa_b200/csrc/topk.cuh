@@ -913,11 +913,12 @@ __global__ void __launch_bounds__(PIPE_THREADS, PIPE_CTAS_PER_SM) topk_pipe_kern
 //    of key offsets above the prediction (bins of 2^15 key steps: one
 //    binade, the last bin taking everything above).  At the end of a row the
 //    histogram gives the bin of its k-th key, so the prediction for the next
-//    row follows every row: 0.85 x the bin's lower edge, kept unchanged while
-//    it stays within 0.75 .. 0.9 of that edge (a CPU replay of the 4 x
-//    4,096-row workload's rows: 0.4% of rows short of k, almost none over a
-//    segment).  A row without a prediction, with fewer than k candidates or
-//    with a full segment is marked for the exact pass.
+//    row follows every row: 0.88 x the bin's lower edge, kept unchanged while
+//    it stays within 0.8 .. 0.93 of that edge (on the 4 x 4,096-row
+//    workload's rows: ~1,200 candidates per row, 1.7% of rows short of k and
+//    none over a segment; 0.85 .. 0.75 .. 0.9 gave 1,480 candidates and 0.4%
+//    short, a little slower overall).  A row without a prediction, with fewer
+//    than k candidates or with a full segment is marked for the exact pass.
 //  * topk_list_kernel: one warp per row, no block barriers: the stored
 //    histogram gives the boundary bin, one pass over the list marks the
 //    columns of higher bins in the warp's column bitmap and sets the boundary
@@ -934,9 +935,9 @@ constexpr int TP_CAP = 4096;          // staged candidates per row (global memor
 constexpr int TP_SEG = TP_CAP / TP_FILT_WARPS;
 constexpr int TP_BINS = 256;
 constexpr int TP_SHIFT = 15;
-constexpr float TP_MARGIN = 0.85f;
-constexpr float TP_KEEP_LO = 0.75f;
-constexpr float TP_KEEP_HI = 0.9f;
+constexpr float TP_MARGIN = 0.88f;
+constexpr float TP_KEEP_LO = 0.8f;
+constexpr float TP_KEEP_HI = 0.93f;
 constexpr uint32_t TP_FILTER_BAR = 1;
 constexpr int TP_LIST_WARPS = 8;
 constexpr int TP_LIST_CTAS_PER_SM = 4;
